@@ -1,0 +1,277 @@
+"""Pins of the fp64 oracle to facts other than the oracle itself.
+
+Each function takes an `oracle.Oracle` and raises AssertionError when the
+oracle disagrees with:
+  * numbers the pages print (worked VSA routing example; 96*64*64 tokens),
+  * a library routine that computes the same thing by another road
+    (numpy reshape-mean, numpy/torch top-k, torch scaled_dot_product_attention
+    with or without a token mask),
+  * brute force on tiny inputs (enumeration of all 2^nb block subsets), or
+  * invariants the method fixes (kept mass >= p, floor, diagonal, ascending,
+    weights summing to one, convex combination).
+The same functions are re-run on deliberately broken copies of the oracle in
+`test_oracle_mutants.py`; every broken copy must fail at least one of them.
+"""
+from __future__ import annotations
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+from block_sparse_attention_fvattn_b200 import inputs as gen
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _token_blocks(grid, block):
+    """Independent token -> block map (numpy, raster order T slowest)."""
+    T, Hg, W = grid
+    bt, bh, bw = block
+    t, y, x = np.meshgrid(np.arange(T), np.arange(Hg), np.arange(W), indexing="ij")
+    nbh, nbw = -(-Hg // bh), -(-W // bw)
+    return ((t // bt) * nbh + (y // bh)) * nbw + (x // bw)
+
+
+def _softmax_rows(s):
+    m = s.max(axis=-1, keepdims=True)
+    e = np.exp(s - m)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def _np_scores(qbar, kbar, scale):
+    return scale * np.einsum("bhid,bhjd->bhij", qbar, kbar)
+
+
+def _small(grid, block, H=2, D=32, sigma=1.5, seed=11, iid=False):
+    if iid:
+        wl = gen.custom("pin", 1, H, D, grid, block, 0.9, 2, seed=seed)
+    else:
+        wl = gen.custom("pin", 1, H, D, grid, block, 0.9, 2, sigma=sigma, a_range=(0.5, 3.0), seed=seed)
+    q, k, v = gen.make_inputs(wl, "cpu")
+    return wl, q, k, v
+
+
+# ---------------------------------------------------------------- geometry
+def pin_vsa_worked_example(orc):
+    ex = _load("vsa_routing_example.json")
+    g = orc.geom(1, 1, ex["dit_seq_shape"], ex["block_size"], 64)
+    nb = orc.num_blocks(g)
+    assert nb == ex["num_blocks"], nb
+    assert int(np.prod(ex["dit_seq_shape"])) == ex["seq_len"]
+    assert round(100.0 * ex["topk"] / nb, 1) == ex["keep_ratio_percent_1dp"]
+    sizes = orc.block_sizes(g)
+    tb = _token_blocks(ex["dit_seq_shape"], ex["block_size"]).ravel()
+    brute = np.bincount(tb, minlength=nb)
+    assert np.array_equal(sizes, brute), "valid token counts per block"
+    assert sizes.sum() == ex["seq_len"]
+
+
+def pin_long_video_tokens(orc):
+    ex = _load("long_video_tokens.json")
+    assert int(np.prod(ex["latent_grid"])) == ex["tokens"]
+    g = orc.geom(1, 1, ex["latent_grid"], (4, 8, 8), 64)
+    assert orc.num_blocks(g) == 24 * 8 * 8
+    assert orc.block_sizes(g).sum() == ex["tokens"]
+    # a token-level bool mask would take n^2 bytes (~155e9, "about 160 GB");
+    # per-(head, query-block) lists take at most 4*nb^2 bytes per head
+    assert abs(ex["tokens"] ** 2 / 1e9 - ex["bool_mask_gb_approx"]) < 0.05 * ex["bool_mask_gb_approx"]
+    assert 4 * orc.num_blocks(g) ** 2 < ex["tokens"] ** 2 / 1000
+
+
+# ---------------------------------------------------------------- pooling
+def pin_pool_reshape_mean(orc):
+    wl, q, k, v = _small((8, 16, 16), (4, 8, 8))
+    g = orc.geom(wl.B, wl.H, wl.grid, wl.block, wl.D)
+    got = orc.pool(g, q)
+    x = q.double().numpy().reshape(1, wl.H, 2, 4, 2, 8, 2, 8, wl.D)
+    ref = x.mean(axis=(3, 5, 7)).reshape(1, wl.H, 8, wl.D)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def pin_pool_ragged_bruteforce(orc):
+    grid, block = (5, 11, 13), (4, 8, 8)
+    wl, q, k, v = _small(grid, block, D=16)
+    g = orc.geom(wl.B, wl.H, grid, block, wl.D)
+    nb = orc.num_blocks(g)
+    got = orc.pool(g, k)
+    tb = _token_blocks(grid, block).ravel()
+    x = k.double().numpy()[0]
+    for h in range(wl.H):
+        sums = np.zeros((nb, wl.D))
+        np.add.at(sums, tb, x[h])
+        cnt = np.bincount(tb, minlength=nb)[:, None]
+        np.testing.assert_allclose(got[0, h], sums / cnt, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- routing
+def _route_small(orc, grid, block, p, k_min, H=2, D=32, iid=True, seed=5):
+    wl, q, k, v = _small(grid, block, H=H, D=D, iid=iid, seed=seed)
+    g = orc.geom(wl.B, wl.H, grid, block, D)
+    qb, kb = orc.pool(g, q), orc.pool(g, k)
+    scale = 1.0 / math.sqrt(D)
+    r = orc.route(g, qb, kb, scale, p, k_min)
+    return wl, g, q, k, v, qb, kb, scale, r
+
+
+def pin_topp_bruteforce(orc):
+    """nb = 8: enumerate all 256 subsets of every row."""
+    grid, block = (8, 16, 16), (4, 8, 8)
+    for p, k_min in [(0.3, 1), (0.5, 1), (0.9, 2), (0.99, 1), (0.75, 5)]:
+        wl, g, q, k, v, qb, kb, scale, r = _route_small(orc, grid, block, p, k_min, D=8, iid=True, seed=3)
+        P = _softmax_rows(_np_scores(qb, kb, scale))
+        nb = P.shape[-1]
+        subsets = [np.array(c, dtype=int) for m in range(1, nb + 1) for c in itertools.combinations(range(nb), m)]
+        for h in range(wl.H):
+            for i in range(nb):
+                row = P[0, h, i]
+                best_m, best_set = None, None
+                for sset in subsets:
+                    mass = row[sset].sum()
+                    if mass >= p and (best_m is None or len(sset) < best_m or
+                                      (len(sset) == best_m and mass > row[best_set].sum())):
+                        best_m, best_set = len(sset), sset
+                m = min(nb, max(best_m, k_min))
+                top_m = max((c for c in subsets if len(c) == m), key=lambda c: row[c].sum())
+                expect = sorted(set(top_m.tolist()) | {i})
+                cnt = r["kv_cnt"][0, h, i]
+                got = r["kv_idx"][0, h, i, :cnt].tolist()
+                assert got == expect, (p, k_min, h, i, got, expect)
+                # the Top-p count read from the oracle's cumulative sums
+                cum = r["cum"][0, h, i]
+                m_p = int(np.argmax(cum >= p)) + 1
+                assert m_p == best_m, (m_p, best_m)
+
+
+def pin_topk_reduction(orc):
+    """p -> 0+ with k_min = k is a fixed top-k (VSA's selection) plus the diagonal."""
+    grid, block = (12, 24, 24), (4, 8, 8)
+    for kk in (1, 3, 7, 18):
+        wl, g, q, k, v, qb, kb, scale, r = _route_small(orc, grid, block, 1e-12, kk, D=32, iid=False)
+        s = _np_scores(qb, kb, scale)
+        nb = s.shape[-1]
+        for h in range(wl.H):
+            for i in range(nb):
+                top = torch.topk(torch.from_numpy(s[0, h, i]), kk).indices.tolist()
+                expect = sorted(set(top) | {i})
+                cnt = r["kv_cnt"][0, h, i]
+                assert r["kv_idx"][0, h, i, :cnt].tolist() == expect, (kk, h, i)
+
+
+def pin_dense_reduction(orc):
+    """p = 1 or k_min = nb keeps every block; attention is then plain softmax
+    attention, checked against torch's scaled_dot_product_attention in fp64."""
+    for grid in [(8, 16, 16), (5, 11, 13)]:
+        block = (4, 8, 8)
+        for p, k_min in [(1.0, 1), (0.5, None)]:
+            wl, q, k, v = _small(grid, block, H=2, D=32)
+            g = orc.geom(wl.B, wl.H, grid, block, wl.D)
+            nb = orc.num_blocks(g)
+            km = nb if k_min is None else k_min
+            qb, kb = orc.pool(g, q), orc.pool(g, k)
+            r = orc.route(g, qb, kb, 1.0 / math.sqrt(wl.D), p, km)
+            assert (r["kv_cnt"] == nb).all()
+            assert (r["kv_idx"] == np.arange(nb)).all()
+            N = wl.N
+            rows = np.arange(wl.H * N)
+            out, ws = orc.attn_rows(g, q, k, v, 1.0 / math.sqrt(wl.D), rows, r["kv_cnt"], r["kv_idx"])
+            ref = torch.nn.functional.scaled_dot_product_attention(q.double(), k.double(), v.double())
+            np.testing.assert_allclose(out.reshape(1, wl.H, N, wl.D), ref.numpy(), rtol=0, atol=1e-12)
+            np.testing.assert_allclose(ws, 1.0, rtol=0, atol=1e-12)
+
+
+def pin_sparse_attention_masked_sdpa(orc):
+    """Attention over a kept list equals SDPA with the token mask the list implies."""
+    grid, block = (6, 13, 10), (4, 8, 8)
+    wl, g, q, k, v, qb, kb, scale, r = _route_small(orc, grid, block, 0.6, 2, H=2, D=16, iid=False)
+    N = wl.N
+    tb = _token_blocks(grid, block).ravel()
+    rows = np.arange(wl.H * N)
+    out, ws = orc.attn_rows(g, q, k, v, scale, rows, r["kv_cnt"], r["kv_idx"])
+    nb = orc.num_blocks(g)
+    for h in range(wl.H):
+        keep = np.zeros((nb, nb), dtype=bool)
+        for i in range(nb):
+            keep[i, r["kv_idx"][0, h, i, :r["kv_cnt"][0, h, i]]] = True
+        mask = torch.from_numpy(keep[tb][:, tb])
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q[0, h].double(), k[0, h].double(), v[0, h].double(), attn_mask=mask, scale=scale)
+        np.testing.assert_allclose(out[h * N:(h + 1) * N], ref.numpy(), rtol=0, atol=1e-12)
+
+
+def pin_invariants(orc):
+    grid, block = (9, 20, 28), (4, 8, 8)
+    for p, k_min in [(0.9, 4), (0.5, 1), (0.97, 10)]:
+        wl, g, q, k, v, qb, kb, scale, r = _route_small(orc, grid, block, p, k_min, H=2, D=32, iid=False)
+        P = _softmax_rows(_np_scores(qb, kb, scale))
+        nb = P.shape[-1]
+        for h in range(wl.H):
+            for i in range(nb):
+                cnt = r["kv_cnt"][0, h, i]
+                lst = r["kv_idx"][0, h, i, :cnt]
+                assert min(k_min, nb) <= cnt <= nb
+                assert i in lst
+                assert np.all(np.diff(lst) > 0)
+                assert P[0, h, i, lst].sum() >= p - 1e-12
+                # minimality: without the floor and the diagonal, dropping the
+                # weakest Top-p block would fall below p
+                cum = r["cum"][0, h, i]
+                m_p = int(np.argmax(cum >= p)) + 1
+                top = np.sort(P[0, h, i])[::-1]
+                assert top[:m_p].sum() >= p - 1e-12 and (m_p == 1 or top[:m_p - 1].sum() < p + 1e-12)
+        rows = np.random.default_rng(0).choice(wl.H * wl.N, size=200, replace=False)
+        out, ws, lo, hi = orc.attn_rows(g, q, k, v, scale, rows, r["kv_cnt"], r["kv_idx"], want_bounds=True)
+        np.testing.assert_allclose(ws, 1.0, rtol=0, atol=1e-12)
+        assert np.all(out >= lo - 1e-12) and np.all(out <= hi + 1e-12)
+
+
+def pin_tie_order(orc):
+    """Equal scores rank the lower block index first: duplicate two key blocks."""
+    grid, block = (4, 16, 16), (4, 8, 8)   # 4 blocks, all full
+    wl, q, k, v = _small(grid, block, H=1, D=8, iid=True, seed=9)
+    tb = _token_blocks(grid, block).ravel()
+    kk = k.clone()
+    kk[0, 0, tb == 3] = kk[0, 0, tb == 1]          # block 3 := block 1 (same mean)
+    g = orc.geom(1, 1, grid, block, 8)
+    qb, kb = orc.pool(g, q), orc.pool(g, kk)
+    assert np.array_equal(kb[0, 0, 1], kb[0, 0, 3])
+    s = _np_scores(qb, kb, 0.5)[0, 0]
+    for i in range(4):
+        # choose k_min so that the floor cuts exactly between the two tied blocks
+        order = sorted(range(4), key=lambda j: (-s[i, j], j))
+        pos = order.index(1)
+        assert order[pos + 1] == 3
+        r = orc.route(g, qb, kb, 0.5, 1e-12, pos + 1)
+        lst = set(r["kv_idx"][0, 0, i, :r["kv_cnt"][0, 0, i]].tolist())
+        assert 1 in lst
+        assert (3 not in lst) or i == 3
+
+
+def pin_nonfinite_repair(orc):
+    grid, block = (8, 16, 16), (4, 8, 8)
+    wl, q, k, v = _small(grid, block, H=2, D=16, iid=True)
+    tb = _token_blocks(grid, block).ravel()
+    qq = q.clone()
+    qq[0, 1, np.where(tb == 5)[0][:3]] = float("inf")
+    g = orc.geom(1, 2, grid, block, 16)
+    qb, kb = orc.pool(g, qq), orc.pool(g, k)
+    r = orc.route(g, qb, kb, 0.25, 0.3, 1)
+    nb = orc.num_blocks(g)
+    assert r["nonfinite"][0, 1, 5] == 1 and r["nonfinite"].sum() == 1
+    assert r["kv_cnt"][0, 1, 5] == nb and (r["kv_idx"][0, 1, 5] == np.arange(nb)).all()
+    assert (r["kv_cnt"][0, 0] < nb).any()
+
+
+ALL_PINS = [
+    pin_vsa_worked_example, pin_long_video_tokens, pin_pool_reshape_mean, pin_pool_ragged_bruteforce,
+    pin_topp_bruteforce, pin_topk_reduction, pin_dense_reduction, pin_sparse_attention_masked_sdpa,
+    pin_invariants, pin_tie_order, pin_nonfinite_repair,
+]
