@@ -1,0 +1,249 @@
+// api.cu -- the extern "C" boundary declared in include/fvattn.h.
+//
+// Validation mirrors the FastVideo VSA backend's acceptance rules (zskr.cn
+// guide, section 5: bf16 tensors, equal Q/K/V head counts, no mask,
+// non-causal equal-length self-attention, a block product of 256 -- or 64 on
+// the (4,4,4) route --, grid product == sequence length; section 3: top-k
+// above num_blocks is rejected, top-k == num_blocks accepted). Where that
+// backend falls back to SDPA, this library returns a status instead: it has
+// no fallback path.
+#include <math.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "fvattn.h"
+#include "internal.h"
+
+namespace fvattn {
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+WsLayout ws_layout(const Geo &g)
+{
+    WsLayout L;
+    size_t off = align256(sizeof(WsHeader));
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align256(off + bytes);
+        return o;
+    };
+    L.qbar = take((size_t)g.BH * g.nb * g.D * sizeof(float));
+    L.kbarT = take((size_t)g.BH * g.D * g.nbp * sizeof(float));
+    L.unit_cost = take((size_t)g.BH * g.nb * sizeof(int32_t));
+    L.head_sorted = take((size_t)g.BH * g.nb * sizeof(int32_t));
+    L.head_cost = take((size_t)g.BH * sizeof(int64_t));
+    L.total = off;
+    return L;
+}
+
+// Resolve and check a problem. Returns FVATTN_OK with *g filled in.
+static fvattn_status resolve(const fvattn_problem *p, Geo *g)
+{
+    if (!p) return FVATTN_ERR_INVALID_ARG;
+    if (p->B < 0 || p->H < 0 || p->N < 1 || p->D < 1) return FVATTN_ERR_INVALID_ARG;
+    if (p->grid_t < 1 || p->grid_h < 1 || p->grid_w < 1) return FVATTN_ERR_INVALID_ARG;
+    if (p->blk_t < 1 || p->blk_h < 1 || p->blk_w < 1) return FVATTN_ERR_INVALID_ARG;
+    if ((long long)p->grid_t * p->grid_h * p->grid_w != (long long)p->N) return FVATTN_ERR_INVALID_ARG;
+    if (isnan(p->softmax_scale) || isinf(p->softmax_scale)) return FVATTN_ERR_INVALID_ARG;
+    if (p->D != 64 && p->D != 128) return FVATTN_ERR_UNSUPPORTED;
+    const long long bp = (long long)p->blk_t * p->blk_h * p->blk_w;
+    if (!(bp == 256 && p->blk_t % 2 == 0) && bp != 64) return FVATTN_ERR_UNSUPPORTED;
+    if (p->blk_w > 256 || p->blk_h > 256 || p->blk_t > 256) return FVATTN_ERR_UNSUPPORTED;
+    Geo G;
+    G.B = p->B;
+    G.H = p->H;
+    G.N = p->N;
+    G.D = p->D;
+    G.T = p->grid_t;
+    G.Hg = p->grid_h;
+    G.W = p->grid_w;
+    G.bt = p->blk_t;
+    G.bh = p->blk_h;
+    G.bw = p->blk_w;
+    G.nbt = ceil_div(G.T, G.bt);
+    G.nbh = ceil_div(G.Hg, G.bh);
+    G.nbw = ceil_div(G.W, G.bw);
+    const long long nb = (long long)G.nbt * G.nbh * G.nbw;
+    if (nb > kMaxBlocks) return FVATTN_ERR_UNSUPPORTED;
+    G.nb = (int)nb;
+    const long long bh = (long long)G.B * G.H;
+    if (bh > 65535) return FVATTN_ERR_UNSUPPORTED;
+    G.BH = (int)bh;
+    G.nbp = (G.nb + 3) & ~3;
+    if (bp == 256) {
+        G.subt = G.bt / 2;
+        G.nsub = 2;
+        G.rows = 128;
+    } else {
+        G.subt = G.bt;
+        G.nsub = 1;
+        G.rows = 64;
+    }
+    G.scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / sqrtf((float)G.D);
+    *g = G;
+    return FVATTN_OK;
+}
+
+static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+static bool aligned4(const void *p) { return ((uintptr_t)p & 3u) == 0; }
+
+static int num_sms()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    return n;
+}
+
+static fvattn_status check_ws(const Geo &g, const void *ws, size_t ws_bytes)
+{
+    if (!ws || !aligned16(ws)) return FVATTN_ERR_WORKSPACE;
+    if (ws_bytes < ws_layout(g).total) return FVATTN_ERR_WORKSPACE;
+    return FVATTN_OK;
+}
+
+}  // namespace fvattn
+
+using namespace fvattn;
+
+extern "C" {
+
+int32_t fvattn_num_blocks(const fvattn_problem *prob)
+{
+    Geo g;
+    if (resolve(prob, &g) != FVATTN_OK) return -1;
+    return g.nb;
+}
+
+int32_t fvattn_default_num_ctas(void) { return num_sms(); }
+
+size_t fvattn_workspace_size(const fvattn_problem *prob, int32_t num_ctas)
+{
+    (void)num_ctas;
+    Geo g;
+    if (resolve(prob, &g) != FVATTN_OK) return 0;
+    return ws_layout(g).total;
+}
+
+fvattn_status fvattn_workspace_init(void *ws, size_t ws_bytes, fvattn_stream_t stream)
+{
+    if (!ws || ws_bytes < sizeof(WsHeader) || !aligned16(ws)) return FVATTN_ERR_WORKSPACE;
+    if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), (cudaStream_t)stream) != cudaSuccess) return FVATTN_ERR_CUDA;
+    return FVATTN_OK;
+}
+
+fvattn_status fvattn_route(const fvattn_problem *prob, const void *q, const void *k, float p, int32_t k_min,
+                           int32_t *kv_cnt, int32_t *kv_idx, float *block_probs, void *ws, size_t ws_bytes,
+                           fvattn_stream_t stream)
+{
+    Geo g;
+    fvattn_status st = resolve(prob, &g);
+    if (st != FVATTN_OK) return st;
+    if (!(p > 0.f && p <= 1.f)) return FVATTN_ERR_INVALID_ARG;  // also rejects NaN
+    if (k_min < 1 || k_min > g.nb) return FVATTN_ERR_INVALID_ARG;
+    if (!q || !k || !aligned16(q) || !aligned16(k)) return FVATTN_ERR_INVALID_ARG;
+    if (!kv_cnt || !kv_idx || !aligned4(kv_cnt) || !aligned4(kv_idx)) return FVATTN_ERR_INVALID_ARG;
+    if (block_probs && !aligned4(block_probs)) return FVATTN_ERR_INVALID_ARG;
+    st = check_ws(g, ws, ws_bytes);
+    if (st != FVATTN_OK) return st;
+    if (g.BH == 0) return FVATTN_OK;
+    const WsLayout L = ws_layout(g);
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    float *qbar = reinterpret_cast<float *>(w + L.qbar);
+    float *kbarT = reinterpret_cast<float *>(w + L.kbarT);
+    uint32_t *status = reinterpret_cast<uint32_t *>(w);
+    cudaStream_t s = (cudaStream_t)stream;
+    if (launch_pool(g, q, k, qbar, kbarT, s) != cudaSuccess) return FVATTN_ERR_CUDA;
+    if (launch_score_select(g, qbar, kbarT, p, k_min, kv_cnt, kv_idx, block_probs, status, s) != cudaSuccess)
+        return FVATTN_ERR_CUDA;
+    return FVATTN_OK;
+}
+
+fvattn_status fvattn_schedule(const fvattn_problem *prob, const int32_t *kv_cnt, const int32_t *kv_idx,
+                              int32_t dense, int32_t num_ctas, int32_t *work, int32_t *cta_range,
+                              int64_t *cta_cost, void *ws, size_t ws_bytes, fvattn_stream_t stream)
+{
+    Geo g;
+    fvattn_status st = resolve(prob, &g);
+    if (st != FVATTN_OK) return st;
+    if (num_ctas < 0 || num_ctas > kMaxCtas) return FVATTN_ERR_INVALID_ARG;
+    if (!dense && (!kv_cnt || !kv_idx)) return FVATTN_ERR_INVALID_ARG;
+    if (!work || !cta_range) return FVATTN_ERR_INVALID_ARG;
+    st = check_ws(g, ws, ws_bytes);
+    if (st != FVATTN_OK) return st;
+    if (num_ctas == 0) {
+        num_ctas = num_sms();
+        if (num_ctas <= 0) return FVATTN_ERR_CUDA;
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    if (g.BH == 0) {
+        if (cudaMemsetAsync(cta_range, 0, sizeof(int32_t) * (size_t)(num_ctas + 1), s) != cudaSuccess)
+            return FVATTN_ERR_CUDA;
+        if (cta_cost && cudaMemsetAsync(cta_cost, 0, sizeof(int64_t) * (size_t)num_ctas, s) != cudaSuccess)
+            return FVATTN_ERR_CUDA;
+        return FVATTN_OK;
+    }
+    const WsLayout L = ws_layout(g);
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    if (launch_schedule(g, kv_cnt, kv_idx, dense ? 1 : 0, num_ctas, work, cta_range, cta_cost,
+                        reinterpret_cast<int32_t *>(w + L.unit_cost), reinterpret_cast<int32_t *>(w + L.head_sorted),
+                        reinterpret_cast<int64_t *>(w + L.head_cost), s) != cudaSuccess)
+        return FVATTN_ERR_CUDA;
+    return FVATTN_OK;
+}
+
+fvattn_status fvattn_sparse_attn(const fvattn_problem *prob, const void *q, const void *k, const void *v,
+                                 const int32_t *kv_cnt, const int32_t *kv_idx, const int32_t *work,
+                                 const int32_t *cta_range, int32_t num_ctas, int32_t dense, void *out,
+                                 int64_t *cta_ns, void *ws, size_t ws_bytes, fvattn_stream_t stream)
+{
+    Geo g;
+    fvattn_status st = resolve(prob, &g);
+    if (st != FVATTN_OK) return st;
+    if (!q || !k || !v || !out) return FVATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return FVATTN_ERR_INVALID_ARG;
+    if (!dense && (!kv_cnt || !kv_idx)) return FVATTN_ERR_INVALID_ARG;
+    if ((work == nullptr) != (cta_range == nullptr)) return FVATTN_ERR_INVALID_ARG;
+    if (num_ctas < 0 || num_ctas > kMaxCtas) return FVATTN_ERR_INVALID_ARG;
+    st = check_ws(g, ws, ws_bytes);
+    if (st != FVATTN_OK) return st;
+    if (num_ctas == 0) {
+        num_ctas = num_sms();
+        if (num_ctas <= 0) return FVATTN_ERR_CUDA;
+    }
+    if (g.BH == 0) return FVATTN_OK;
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+    int kind = 0;
+    if (launch_attn(g, q, k, v, kv_cnt, kv_idx, work, cta_range, num_ctas, dense ? 1 : 0, out, cta_ns, status,
+                    (cudaStream_t)stream, &kind) != cudaSuccess)
+        return FVATTN_ERR_CUDA;
+    return FVATTN_OK;
+}
+
+fvattn_status fvattn_read_device_status(void *ws, fvattn_stream_t stream, uint32_t *flags)
+{
+    if (!ws || !flags) return FVATTN_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint32_t host = 0;
+    if (cudaMemcpyAsync(&host, ws, sizeof(uint32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess) return FVATTN_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return FVATTN_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return FVATTN_ERR_CUDA;
+    *flags = host;
+    return FVATTN_OK;
+}
+
+const char *fvattn_status_string(fvattn_status s)
+{
+    switch (s) {
+    case FVATTN_OK: return "ok";
+    case FVATTN_ERR_INVALID_ARG: return "invalid argument";
+    case FVATTN_ERR_UNSUPPORTED: return "unsupported problem shape";
+    case FVATTN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case FVATTN_ERR_CUDA: return "CUDA call failed";
+    case FVATTN_STATUS_NONFINITE: return "non-finite block scores were repaired";
+    case FVATTN_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,623 @@
+// attn.cu -- K4: persistent block-sparse attention on sm_100a (TMA + tcgen05/TMEM).
+//
+// Attention runs only over the key/value blocks kept by the router (the
+// source of the method's attention speedup over FlashAttention: ai-feeds.com
+// FVAttn summary, "Key findings"; zskr.cn FastVideo VSA guide, section 1:
+// each query block attends to its selected key/value blocks). Dense mode
+// runs every block through the same code (the guide's VSA_ALL_BLOCKS route).
+//
+// Work unit = one (b, h, query block i). A 256-token block is two 128-row
+// query tiles (its two halves along t), a 64-token block one 64-row tile.
+// Key/value blocks are consumed in sub-tiles of 128 (or 64) tokens, so one
+// 256-token key block is two sub-tiles; a sub-tile that lies wholly outside
+// the grid is skipped, partial ones mask their padded columns.
+//
+// Tiles come straight from the raster [B,H,N,D] layout: each tensor is seen
+// by TMA as 5-D (D, W, H, T, B*H) and one sub-tile is one box of
+// (64, bw, bh, sub_t, 1) elements per 64-column slab, 128-byte swizzled.
+// Out-of-grid elements are filled with zeros by TMA; no token-level mask or
+// re-packed copy of the sequence is ever built (the bjdmk.com.cn Sol-Attn
+// article, section 5.1, on n x n masks at ~400k tokens).
+//
+// Roles (384 threads = 3 warpgroups, one CTA per SM):
+//   warp 0      TMA producer: Q halves, K and V sub-tiles into rings
+//   warp 1      MMA issuer: S_h = Q_h K^T (A, B from shared memory) and
+//               O_h += P_h V (A = P from tensor memory, B = V from shared
+//               memory, MN-major); owns the TMEM allocation
+//   warps 2-3   idle (they only return registers)
+//   warps 4-7   softmax + epilogue for query half 0
+//   warps 8-11  softmax + epilogue for query half 1
+// A warp reaches TMEM lanes 32*(warp % 4) .. +31, so each softmax warpgroup
+// covers the 128 rows of its half (row = 32*(warp%4) + lane) and holds a
+// whole 128-column score row in registers.
+// TMEM columns: S_0 [0,128) S_1 [128,256) O_0 [256,256+D) O_1 [256+D, 256+2D);
+// P_h (bf16 pairs) overwrites the first BKV/2 columns of S_h. The online
+// softmax rescales O lazily, only when a row maximum grows by more than 2^8.
+#include "common.cuh"
+#include "internal.h"
+
+namespace fvattn {
+
+constexpr int kNK = 2;  // K ring stages
+constexpr int kNV = 2;  // V ring stages
+constexpr int kThreads = 384;
+// Register split between warpgroups (setmaxnreg). The kernel is launched with
+// kLaunchRegs per thread (checked on the host before every launch); the
+// producer/MMA warpgroup gives registers back and the two softmax
+// warpgroups take them: 128*kRegsLow + 256*kRegsHigh == 384*kLaunchRegs.
+constexpr int kLaunchRegs = 168;
+constexpr int kRegsLow = 56;
+constexpr int kRegsHigh = 224;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kLaunchRegs, "register split exceeds the launch budget");
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D, int BKV>
+struct AttnLayout {
+    static constexpr int kDH = D / 64;              // 128-byte column slabs per row
+    static constexpr int kQSlab = 128 * 128;        // bytes of one 128-row slab
+    static constexpr int kKVSlab = BKV * 128;
+    static constexpr int kQ = 0;
+    static constexpr int kK = kQ + 2 * kDH * kQSlab;
+    static constexpr int kV = kK + kNK * kDH * kKVSlab;
+    static constexpr int kMask = kV + kNV * kDH * kKVSlab;
+    static constexpr int kMaskWords = BKV / 32;
+    static constexpr int kBar = kMask + BKV * kMaskWords * 4;
+    // barrier indices
+    static constexpr int bQFull = 0, bQEmpty = 2, bKFull = 4, bKEmpty = bKFull + kNK, bVFull = bKEmpty + kNK,
+                         bVEmpty = bVFull + kNV, bSFull = bVEmpty + kNV, bPFull = bSFull + 2, bOFull = bPFull + 2,
+                         bOEmpty = bOFull + 2, bPVDone = bOEmpty + 2, bDrain = bPVDone + 2, kNumBars = bDrain + 1;
+    static constexpr int kMisc = kBar + kNumBars * 8;
+    static constexpr int kBytes = kMisc + 64;
+    static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
+};
+
+struct Unit {
+    int bh, i, it, iy, ix, nh, cnt, nkv;
+    const int32_t *list;
+};
+
+__device__ __forceinline__ Unit load_unit(const Geo &g, int u, const int32_t *kv_cnt, const int32_t *kv_idx,
+                                          int dense)
+{
+    Unit U;
+    U.bh = u / g.nb;
+    U.i = u - U.bh * g.nb;
+    const int hw = g.nbh * g.nbw;
+    U.it = U.i / hw;
+    U.iy = (U.i / g.nbw) % g.nbh;
+    U.ix = U.i % g.nbw;
+    U.nh = (g.nsub == 2 && U.it * g.bt + g.subt < g.T) ? 2 : 1;
+    U.cnt = dense ? g.nb : __ldg(kv_cnt + u);
+    U.list = dense ? nullptr : kv_idx + (size_t)u * g.nb;
+    const bool last_short = (g.nsub == 2) && ((g.nbt - 1) * g.bt + g.subt >= g.T);
+    int nlast = 0;
+    if (last_short) {
+        const int j0 = (g.nbt - 1) * hw;
+        if (dense) {
+            nlast = g.nb - j0;
+        } else {
+            int lo = 0, hi = U.cnt;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (__ldg(U.list + mid) >= j0) hi = mid;
+                else lo = mid + 1;
+            }
+            nlast = U.cnt - lo;
+        }
+    }
+    U.nkv = U.cnt * g.nsub - nlast;
+    return U;
+}
+
+// Walks the kept sub-tiles of a unit in list order.
+struct TileCursor {
+    int e = 0, s = 0;
+    __device__ __forceinline__ int block(const Unit &U) const { return U.list ? __ldg(U.list + e) : e; }
+    __device__ __forceinline__ void advance(const Geo &g, const Unit &U)
+    {
+        if (g.nsub == 2 && s == 0) {
+            const int jt = block(U) / (g.nbh * g.nbw);
+            if (jt * g.bt + g.subt < g.T) {
+                s = 1;
+                return;
+            }
+        }
+        s = 0;
+        ++e;
+    }
+};
+
+// Units of CTA c: either its slice of the scheduled work list, or (no list)
+// the round-robin sequence c, c + C, c + 2C, ...
+struct UnitSeq {
+    const int32_t *work;
+    long long begin, end;
+    long long stride, total;
+    __device__ __forceinline__ bool get(long long idx, int &u) const
+    {
+        if (work) {
+            if (begin + idx >= end) return false;
+            u = __ldg(work + begin + idx);
+            return true;
+        }
+        const long long v = begin + idx * stride;
+        if (v >= total) return false;
+        u = (int)v;
+        return true;
+    }
+};
+
+template <int D, int BKV>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, Geo g, const int32_t *__restrict__ kv_cnt,
+                const int32_t *__restrict__ kv_idx, const int32_t *__restrict__ work,
+                const int32_t *__restrict__ cta_range, int dense, __nv_bfloat16 *__restrict__ out,
+                int64_t *__restrict__ cta_ns, uint32_t *__restrict__ status)
+{
+    using L = AttnLayout<D, BKV>;
+    extern __shared__ uint8_t attn_smem_raw[];
+    const uint32_t raw = smem_u32(attn_smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    uint8_t *gbase = attn_smem_raw + (sbase - raw);
+    const uint32_t *mask_tab = reinterpret_cast<const uint32_t *>(gbase + L::kMask);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + L::kMisc);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + L::kMisc + 16);
+    auto bar = [&](int idx) -> uint32_t { return sbase + L::kBar + 8u * (uint32_t)idx; };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint64_t t_start = globaltimer_ns();
+
+    // ---- set-up: column-validity table, barriers, TMEM
+    {
+        uint32_t *tab = reinterpret_cast<uint32_t *>(gbase + L::kMask);
+        for (int pat = threadIdx.x; pat < BKV; pat += blockDim.x) {
+            const int wv = pat % g.bw + 1, hv = (pat / g.bw) % g.bh + 1, tv = pat / (g.bw * g.bh) + 1;
+            for (int w = 0; w < L::kMaskWords; ++w) {
+                uint32_t word = 0;
+                for (int b = 0; b < 32; ++b) {
+                    const int c = w * 32 + b;
+                    const int tt = c / (g.bh * g.bw), yy = (c / g.bw) % g.bh, xx = c % g.bw;
+                    if (xx < wv && yy < hv && tt < tv) word |= 1u << b;
+                }
+                tab[pat * L::kMaskWords + w] = word;
+            }
+        }
+    }
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        for (int b = 0; b < L::kNumBars; ++b) {
+            uint32_t cnt = 1;
+            if (b == L::bPFull || b == L::bPFull + 1 || b == L::bOEmpty || b == L::bOEmpty + 1) cnt = 128;
+            mbar_init(bar(b), cnt);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    UnitSeq seq;
+    seq.work = work;
+    if (work) {
+        seq.begin = __ldg(cta_range + blockIdx.x);
+        seq.end = __ldg(cta_range + blockIdx.x + 1);
+    } else {
+        seq.begin = blockIdx.x;
+        seq.end = 0;
+    }
+    seq.stride = gridDim.x;
+    seq.total = (long long)g.BH * g.nb;
+
+    constexpr uint32_t kTileBytes = (uint32_t)L::kDH * BKV * 128u;
+    const uint32_t q_bytes = (uint32_t)L::kDH * (uint32_t)g.rows * 128u;
+
+    if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+    if (warp == 0) {
+        // ================= TMA producer =================
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            int kc = 0, vc = 0;
+            uint32_t q_par = 0, q_used = 0;  // per half: loads issued & 1, any load issued
+            bool ok = true;
+            int u;
+            for (long long idx = 0; ok && seq.get(idx, u); ++idx) {
+                const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
+                const int x0 = U.ix * g.bw, y0 = U.iy * g.bh, t0 = U.it * g.bt;
+                for (int h = 0; h < U.nh && ok; ++h) {
+                    if (((q_used >> h) & 1u) &&
+                        !mbar_wait(bar(L::bQEmpty + h), ((q_par >> h) & 1u) ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(bar(L::bQFull + h), q_bytes);
+                    for (int dh = 0; dh < L::kDH; ++dh)
+                        tma_load_5d(sbase + L::kQ + (h * L::kDH + dh) * L::kQSlab, &tm_q, bar(L::bQFull + h),
+                                    dh * 64, x0, y0, t0 + h * g.subt, U.bh);
+                    q_par ^= 1u << h;
+                    q_used |= 1u << h;
+                }
+                TileCursor cur;
+                for (int k = 0; k < U.nkv && ok; ++k) {
+                    const int j = cur.block(U);
+                    const int jt = j / (g.nbh * g.nbw), jy = (j / g.nbw) % g.nbh, jx = j % g.nbw;
+                    const int tt0 = jt * g.bt + cur.s * g.subt;
+                    const int ks = kc % kNK;
+                    if (kc >= kNK && !mbar_wait(bar(L::bKEmpty + ks), ((kc / kNK) - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(bar(L::bKFull + ks), kTileBytes);
+                    for (int dh = 0; dh < L::kDH; ++dh)
+                        tma_load_5d(sbase + L::kK + (ks * L::kDH + dh) * L::kKVSlab, &tm_k, bar(L::bKFull + ks),
+                                    dh * 64, jx * g.bw, jy * g.bh, tt0, U.bh);
+                    ++kc;
+                    const int vs = vc % kNV;
+                    if (vc >= kNV && !mbar_wait(bar(L::bVEmpty + vs), ((vc / kNV) - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(bar(L::bVFull + vs), kTileBytes);
+                    for (int dh = 0; dh < L::kDH; ++dh)
+                        tma_load_5d(sbase + L::kV + (vs * L::kDH + dh) * L::kKVSlab, &tm_v, bar(L::bVFull + vs),
+                                    dh * 64, jx * g.bw, jy * g.bh, tt0, U.bh);
+                    ++vc;
+                    cur.advance(g, U);
+                }
+            }
+            if (!ok) {
+                // wind down: let every copy already issued land before the CTA exits
+                for (int s = 0; s < kNK; ++s) {
+                    const int n = (kc > s) ? (kc - s + kNK - 1) / kNK : 0;
+                    if (n > 0) mbar_wait_for(bar(L::bKFull + s), (n - 1) & 1, 50000000ull);
+                }
+                for (int s = 0; s < kNV; ++s) {
+                    const int n = (vc > s) ? (vc - s + kNV - 1) / kNV : 0;
+                    if (n > 0) mbar_wait_for(bar(L::bVFull + s), (n - 1) & 1, 50000000ull);
+                }
+                for (int h = 0; h < 2; ++h)
+                    if ((q_used >> h) & 1u) mbar_wait_for(bar(L::bQFull + h), ((q_par >> h) & 1u) ^ 1u, 50000000ull);
+            }
+        }
+    } else if (warp == 1) {
+        // ================= MMA issuer =================
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16(128, BKV, false);
+            constexpr uint32_t idesc_pv = idesc_bf16(128, D, true);
+            int kc = 0, vc = 0;
+            // one parity bit per query half for each barrier pair, and one
+            // "committed but not yet waited for" bit per half
+            uint32_t ph_q = 0, ph_p = 0, ph_pv = 0, ph_oe = 0, pv_pend = 0, o_pend = 0;
+            bool ok = true;
+            // S_h = Q_h K^T over D in K=16 steps; Q and K slabs are K-major, 128B swizzle
+            auto issue_qk = [&](int h, int ks) {
+                const uint32_t d_tmem = tmem + (uint32_t)(h * 128);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int dh = kk >> 2, within = kk & 3;
+                    const uint32_t a = sbase + L::kQ + (h * L::kDH + dh) * L::kQSlab + within * 32;
+                    const uint32_t b = sbase + L::kK + (ks * L::kDH + dh) * L::kKVSlab + within * 32;
+                    umma_ss(d_tmem, sdesc_sw128(a, 16, 1024), sdesc_sw128(b, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+                }
+            };
+            // O_h (+)= P_h V over the sub-tile in K=16 steps; P from TMEM, V MN-major
+            auto issue_pv = [&](int h, int vs, bool accumulate) {
+                const uint32_t d_tmem = tmem + 256u + (uint32_t)(h * D);
+#pragma unroll
+                for (int kk = 0; kk < BKV / 16; ++kk) {
+                    const uint32_t a_tmem = tmem + (uint32_t)(h * 128 + kk * 8);
+                    const uint32_t b = sbase + L::kV + (vs * L::kDH) * L::kKVSlab + kk * 16 * 128;
+                    umma_ts(d_tmem, a_tmem, sdesc_sw128(b, L::kKVSlab, 1024), idesc_pv,
+                            (accumulate || kk > 0) ? 1u : 0u);
+                }
+            };
+            auto wait_half = [&](int base, uint32_t &ph, int h) -> bool {
+                const bool r = mbar_wait(bar(base + h), (ph >> h) & 1u, abort_flag);
+                ph ^= 1u << h;
+                return r;
+            };
+            int u;
+            for (long long idx = 0; ok && seq.get(idx, u); ++idx) {
+                const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
+                for (int h = 0; h < U.nh && ok; ++h) ok = wait_half(L::bQFull, ph_q, h);
+                if (!ok) break;
+                // first S tiles
+                int ks = kc % kNK;
+                if (!mbar_wait(bar(L::bKFull + ks), (kc / kNK) & 1, abort_flag)) break;
+                tc_fence_after();
+                for (int h = 0; h < U.nh && ok; ++h) {
+                    if ((pv_pend >> h) & 1u) {  // S_h is free once the last PV that read P_h is done
+                        ok = wait_half(L::bPVDone, ph_pv, h);
+                        pv_pend &= ~(1u << h);
+                        tc_fence_after();
+                    }
+                    if (!ok) break;
+                    issue_qk(h, ks);
+                    umma_commit(bar(L::bSFull + h));
+                }
+                if (!ok) break;
+                umma_commit(bar(L::bKEmpty + ks));
+                ++kc;
+                if (U.nkv == 1)
+                    for (int h = 0; h < U.nh; ++h) umma_commit(bar(L::bQEmpty + h));
+                for (int k = 0; k < U.nkv && ok; ++k) {
+                    const int vs = vc % kNV;
+                    if (!mbar_wait(bar(L::bVFull + vs), (vc / kNV) & 1, abort_flag)) { ok = false; break; }
+                    for (int h = 0; h < U.nh && ok; ++h) {
+                        ok = wait_half(L::bPFull, ph_p, h);
+                        if (ok && k == 0 && ((o_pend >> h) & 1u)) {  // previous unit's epilogue read O_h
+                            ok = wait_half(L::bOEmpty, ph_oe, h);
+                            o_pend &= ~(1u << h);
+                        }
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(h, vs, k > 0);
+                        umma_commit(bar(L::bPVDone + h));
+                        pv_pend |= 1u << h;
+                        if (k == U.nkv - 1) {
+                            umma_commit(bar(L::bOFull + h));
+                            o_pend |= 1u << h;
+                        }
+                    }
+                    if (!ok) break;
+                    umma_commit(bar(L::bVEmpty + vs));
+                    ++vc;
+                    if (k + 1 < U.nkv) {
+                        ks = kc % kNK;
+                        if (!mbar_wait(bar(L::bKFull + ks), (kc / kNK) & 1, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                        for (int h = 0; h < U.nh && ok; ++h) {
+                            ok = wait_half(L::bPVDone, ph_pv, h);
+                            pv_pend &= ~(1u << h);
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_qk(h, ks);
+                            umma_commit(bar(L::bSFull + h));
+                        }
+                        if (!ok) break;
+                        umma_commit(bar(L::bKEmpty + ks));
+                        ++kc;
+                        if (k + 2 == U.nkv)
+                            for (int h = 0; h < U.nh; ++h) umma_commit(bar(L::bQEmpty + h));
+                    }
+                }
+            }
+            // every MMA issued must finish before TMEM is released
+            umma_commit(bar(L::bDrain));
+            mbar_wait_for(bar(L::bDrain), 0, 100000000ull);
+        }
+    } else if (warp >= 4) {
+        // ================= softmax + epilogue =================
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
+        const int h = (warp - 4) >> 2;
+        const int wq = warp & 3;
+        const int row = wq * 32 + lane;
+        const uint32_t t_lane = (uint32_t)(wq * 32) << 16;
+        const uint32_t tS = tmem + t_lane + (uint32_t)(h * 128);
+        const uint32_t tO = tmem + t_lane + 256u + (uint32_t)(h * D);
+        const float sl2 = g.scale * 1.4426950408889634f;
+        // this thread's query row inside a sub-tile
+        const int r_t = row / (g.bh * g.bw), r_y = (row / g.bw) % g.bh, r_x = row % g.bw;
+        int sf = 0, of = 0;
+        bool ok = true;
+        int u;
+        for (long long idx = 0; ok && seq.get(idx, u); ++idx) {
+            const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
+            if (h >= U.nh) continue;
+            const int qt = U.it * g.bt + h * g.subt + r_t, qy = U.iy * g.bh + r_y, qx = U.ix * g.bw + r_x;
+            const bool row_valid = row < g.rows && qt < g.T && qy < g.Hg && qx < g.W;
+            float m = -INFINITY, l = 0.f;
+            TileCursor cur;
+            for (int k = 0; k < U.nkv; ++k) {
+                const int j = cur.block(U);
+                const int jt = j / (g.nbh * g.nbw), jy = (j / g.nbw) % g.nbh, jx = j % g.nbw;
+                const int wv = min(g.bw, g.W - jx * g.bw), hv = min(g.bh, g.Hg - jy * g.bh);
+                const int tv = min(g.subt, g.T - (jt * g.bt + cur.s * g.subt));
+                const bool full = (wv == g.bw) && (hv == g.bh) && (tv == g.subt);
+                if (!mbar_wait(bar(L::bSFull + h), sf & 1, abort_flag)) { ok = false; break; }
+                ++sf;
+                tc_fence_after();
+                float x[BKV];
+#pragma unroll
+                for (int c = 0; c < BKV / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tS + c * 32, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int v = 0; v < 32; ++v) x[c * 32 + v] = __uint_as_float(r[v]);
+                }
+                if (!full) {
+                    const uint32_t *mw = mask_tab + (((tv - 1) * g.bh + (hv - 1)) * g.bw + (wv - 1)) * L::kMaskWords;
+#pragma unroll
+                    for (int w = 0; w < L::kMaskWords; ++w) {
+                        const uint32_t word = mw[w];
+#pragma unroll
+                        for (int b = 0; b < 32; ++b)
+                            if (!((word >> b) & 1u)) x[w * 32 + b] = -INFINITY;
+                    }
+                }
+                float mx = x[0];
+#pragma unroll
+                for (int c = 1; c < BKV; ++c) mx = fmaxf(mx, x[c]);
+                const float mt = mx * sl2;
+                float alpha = 1.0f;
+                bool rescale = false;
+                if (k == 0) {
+                    m = mt;
+                } else {
+                    const bool need = mt > m + kRescaleThreshold;
+                    rescale = __any_sync(0xFFFFFFFFu, need);
+                    if (need) {
+                        alpha = ex2_approx(m - mt);
+                        m = mt;
+                        l *= alpha;
+                    }
+                }
+                float sum = 0.f;
+#pragma unroll
+                for (int c = 0; c < BKV / 32; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int q2 = 0; q2 < 16; ++q2) {
+                        const float p0 = ex2_approx(fmaf(x[c * 32 + 2 * q2], sl2, -m));
+                        const float p1 = ex2_approx(fmaf(x[c * 32 + 2 * q2 + 1], sl2, -m));
+                        sum += p0 + p1;
+                        pk[q2] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(tS + c * 16, pk);
+                }
+                if (rescale) {
+                    // O_h holds the sum up to the previous sub-tile (its PV finished
+                    // before this S was produced); bring it to the new row maximum.
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + c * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int v = 0; v < 32; ++v) o[v] = __float_as_uint(__uint_as_float(o[v]) * alpha);
+                        tmem_st32(tO + c * 32, o);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(L::bPFull + h));
+                l += sum;
+                cur.advance(g, U);
+            }
+            if (!ok) break;
+            // epilogue: O / l -> bf16, raster order, valid rows only
+            if (!mbar_wait(bar(L::bOFull + h), of & 1, abort_flag)) { ok = false; break; }
+            ++of;
+            tc_fence_after();
+            const float inv = 1.0f / l;
+            __nv_bfloat16 *orow =
+                out + ((size_t)U.bh * g.N + ((size_t)qt * g.Hg + qy) * g.W + qx) * (size_t)D;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tO + c * 32, o);
+                tmem_wait_ld();
+                if (row_valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(o[q4 * 8 + 0]) * inv, __uint_as_float(o[q4 * 8 + 1]) * inv);
+                        w.y = pack_bf16x2(__uint_as_float(o[q4 * 8 + 2]) * inv, __uint_as_float(o[q4 * 8 + 3]) * inv);
+                        w.z = pack_bf16x2(__uint_as_float(o[q4 * 8 + 4]) * inv, __uint_as_float(o[q4 * 8 + 5]) * inv);
+                        w.w = pack_bf16x2(__uint_as_float(o[q4 * 8 + 6]) * inv, __uint_as_float(o[q4 * 8 + 7]) * inv);
+                        dst[q4] = w;
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar(L::bOEmpty + h));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+    if (threadIdx.x == 0) {
+        if (*abort_flag) atomicOr(status, kFlagTimeout);
+        if (cta_ns) cta_ns[blockIdx.x] = (int64_t)(globaltimer_ns() - t_start);
+    }
+}
+
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// [B*H, T, Hg, W, D] bf16 as a 5-D TMA tensor; box = one sub-tile slab.
+static bool make_map(CUtensorMap *map, const Geo &g, const void *ptr)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[5] = {(cuuint64_t)g.D, (cuuint64_t)g.W, (cuuint64_t)g.Hg, (cuuint64_t)g.T,
+                                (cuuint64_t)g.BH};
+    const cuuint64_t es = 2;
+    const cuuint64_t strides[4] = {(cuuint64_t)g.D * es, (cuuint64_t)g.W * g.D * es,
+                                   (cuuint64_t)g.Hg * g.W * g.D * es, (cuuint64_t)g.N * g.D * es};
+    const cuuint32_t box[5] = {64u, (cuuint32_t)g.bw, (cuuint32_t)g.bh, (cuuint32_t)g.subt, 1u};
+    const cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(ptr), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D, int BKV>
+static cudaError_t launch_attn_t(const Geo &g, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                                 const int32_t *kv_cnt, const int32_t *kv_idx, const int32_t *work,
+                                 const int32_t *cta_range, int grid, int dense, void *out, int64_t *cta_ns,
+                                 uint32_t *status, cudaStream_t stream)
+{
+    using L = AttnLayout<D, BKV>;
+    auto kern = attn_kernel<D, BKV>;
+    cudaFuncAttributes fa;
+    cudaError_t err = cudaFuncGetAttributes(&fa, kern);
+    if (err != cudaSuccess) return err;
+    // the setmaxnreg split must fit in what the launch provides, or the
+    // softmax warpgroups would wait for registers forever
+    if (fa.numRegs * kThreads < 128 * kRegsLow + 256 * kRegsHigh) return cudaErrorInvalidConfiguration;
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (err != cudaSuccess) return err;
+    kern<<<grid, kThreads, L::kAlloc, stream>>>(mq, mk, mv, g, kv_cnt, kv_idx, work, cta_range, dense,
+                                                (__nv_bfloat16 *)out, cta_ns, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attn(const Geo &g, const void *q, const void *k, const void *v, const int32_t *kv_cnt,
+                        const int32_t *kv_idx, const int32_t *work, const int32_t *cta_range, int num_ctas,
+                        int dense, void *out, int64_t *cta_ns, uint32_t *status, cudaStream_t stream,
+                        int *launch_error_kind)
+{
+    *launch_error_kind = 0;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, g, q) || !make_map(&mk, g, k) || !make_map(&mv, g, v)) {
+        *launch_error_kind = 1;
+        return cudaErrorInvalidValue;
+    }
+    int grid = num_ctas;
+    if (!work) {
+        const long long U = (long long)g.BH * g.nb;
+        if (U < grid) grid = (int)U;
+    }
+    if (g.rows == 128) {
+        if (g.D == 128)
+            return launch_attn_t<128, 128>(g, mq, mk, mv, kv_cnt, kv_idx, work, cta_range, grid, dense, out, cta_ns,
+                                           status, stream);
+        return launch_attn_t<64, 128>(g, mq, mk, mv, kv_cnt, kv_idx, work, cta_range, grid, dense, out, cta_ns,
+                                      status, stream);
+    }
+    if (g.D == 128)
+        return launch_attn_t<128, 64>(g, mq, mk, mv, kv_cnt, kv_idx, work, cta_range, grid, dense, out, cta_ns,
+                                      status, stream);
+    return launch_attn_t<64, 64>(g, mq, mk, mv, kv_cnt, kv_idx, work, cta_range, grid, dense, out, cta_ns, status,
+                                 stream);
+}
+
+}  // namespace fvattn

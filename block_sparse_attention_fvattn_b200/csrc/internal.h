@@ -1,0 +1,40 @@
+// internal.h -- launchers shared between the C-ABI shim and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace fvattn {
+
+// Workspace carve-up (byte offsets from the workspace base; 256-byte aligned).
+struct WsLayout {
+    size_t qbar;         // fp32 [BH, nb, D]   pooled query means
+    size_t kbarT;        // fp32 [BH, D, nbp]  pooled key means, transposed
+    size_t unit_cost;    // int32 [BH*nb]      scheduler: cost per unit
+    size_t head_sorted;  // int32 [BH*nb]      scheduler: units of each head by cost
+    size_t head_cost;    // int64 [BH]         scheduler: total cost per head
+    size_t total;
+};
+WsLayout ws_layout(const Geo &g);
+
+// Largest nb the select kernel keeps in registers.
+constexpr int kMaxBlocks = 2048;
+// Largest persistent-CTA count.
+constexpr int kMaxCtas = 4096;
+
+cudaError_t launch_pool(const Geo &g, const void *q, const void *k, float *qbar, float *kbarT,
+                        cudaStream_t stream);
+cudaError_t launch_score_select(const Geo &g, const float *qbar, const float *kbarT, float p, int k_min,
+                                int32_t *kv_cnt, int32_t *kv_idx, float *probs, uint32_t *status,
+                                cudaStream_t stream);
+cudaError_t launch_schedule(const Geo &g, const int32_t *kv_cnt, const int32_t *kv_idx, int dense, int num_ctas,
+                            int32_t *work, int32_t *cta_range, int64_t *cta_cost, int32_t *unit_cost,
+                            int32_t *head_sorted, int64_t *head_cost, cudaStream_t stream);
+cudaError_t launch_attn(const Geo &g, const void *q, const void *k, const void *v, const int32_t *kv_cnt,
+                        const int32_t *kv_idx, const int32_t *work, const int32_t *cta_range, int num_ctas,
+                        int dense, void *out, int64_t *cta_ns, uint32_t *status, cudaStream_t stream,
+                        int *launch_error_kind);
+
+}  // namespace fvattn

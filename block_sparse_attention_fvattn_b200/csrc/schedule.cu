@@ -1,0 +1,180 @@
+// schedule.cu -- longest-first balanced work lists for the persistent attention CTAs.
+//
+// The method observes that Top-p routing leaves heads with very different
+// amounts of kept work, so whoever holds the heaviest heads sets the critical
+// path (ai-feeds.com FVAttn summary, "Existing limitations" and "Key modules"
+// 2; load imbalance = max/mean, ideal 1.0). Its remedy moves heavy heads
+// between GPUs. On one GPU the same imbalance appears between persistent CTAs,
+// and the remedy here is an ordering + assignment:
+//   K3a sched_head_kernel  one CTA per head: cost of every (head, query block)
+//       unit = active 128-row query tiles x kept key/value sub-tiles (what the
+//       attention kernel executes), sorted by cost descending (ties: lower
+//       block index), plus the head's total.
+//   K3b sched_assign_kernel one CTA: heads sorted by total cost descending
+//       (ties: lower head), concatenated into one ranked list; rank r goes to
+//       CTA zigzag(r) (round r/C, direction alternating per round), so every
+//       round of C consecutive ranks -- mostly one head, which keeps its key
+//       and value blocks in L2 -- hands each CTA one unit.
+#include "common.cuh"
+#include "internal.h"
+
+namespace fvattn {
+
+__device__ void bitonic_sort_u64(unsigned long long *keys, int n)
+{
+    for (int k = 2; k <= n; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int t = threadIdx.x; t < n; t += blockDim.x) {
+                const int ixj = t ^ j;
+                if (ixj > t) {
+                    const bool up = (t & k) == 0;
+                    const unsigned long long a = keys[t], b = keys[ixj];
+                    if ((a > b) == up) {
+                        keys[t] = b;
+                        keys[ixj] = a;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+}
+
+// Kept key/value sub-tiles of a unit: every kept block has nsub sub-tiles,
+// except blocks in the last row of t-blocks when its second sub-tile lies
+// wholly outside the grid. Kept lists are ascending, so those blocks are the
+// list's tail, found by binary search.
+__device__ __forceinline__ int unit_tiles(const Geo &g, const int32_t *lst, int cnt, int dense)
+{
+    const bool last_short = (g.nsub == 2) && ((g.nbt - 1) * g.bt + g.subt >= g.T);
+    if (!last_short) return cnt * g.nsub;
+    const int j0 = (g.nbt - 1) * g.nbh * g.nbw;
+    int nlast;
+    if (dense) {
+        nlast = g.nb - j0;
+    } else {
+        int lo = 0, hi = cnt;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldg(lst + mid) >= j0) hi = mid;
+            else lo = mid + 1;
+        }
+        nlast = cnt - lo;
+    }
+    return cnt * g.nsub - nlast;
+}
+
+__global__ void __launch_bounds__(1024) sched_head_kernel(Geo g, const int32_t *__restrict__ kv_cnt,
+                                                          const int32_t *__restrict__ kv_idx, int dense,
+                                                          int32_t *__restrict__ unit_cost,
+                                                          int32_t *__restrict__ head_sorted,
+                                                          int64_t *__restrict__ head_cost, int npow2)
+{
+    extern __shared__ unsigned long long keys[];
+    __shared__ long long part[32];
+    const int bh = blockIdx.x;
+    const int hw = g.nbh * g.nbw;
+    long long local = 0;
+    for (int i = threadIdx.x; i < npow2; i += blockDim.x) {
+        if (i < g.nb) {
+            const size_t u = (size_t)bh * g.nb + i;
+            const int it = i / hw;
+            const int nh = (g.nsub == 2 && it * g.bt + g.subt < g.T) ? 2 : 1;
+            const int cnt = dense ? g.nb : __ldg(kv_cnt + u);
+            const int tiles = unit_tiles(g, dense ? nullptr : kv_idx + u * g.nb, cnt, dense);
+            const int cost = nh * tiles;
+            unit_cost[u] = cost;
+            local += cost;
+            keys[i] = ((unsigned long long)(0xFFFFFFFFu - (uint32_t)cost) << 32) | (uint32_t)i;
+        } else {
+            keys[i] = ~0ull;
+        }
+    }
+    for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xFFFFFFFFu, local, o);
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = local;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        long long s = 0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) s += part[w];
+        head_cost[bh] = s;
+    }
+    bitonic_sort_u64(keys, npow2);
+    for (int r = threadIdx.x; r < g.nb; r += blockDim.x)
+        head_sorted[(size_t)bh * g.nb + r] = (int32_t)(keys[r] & 0xFFFFFFFFull);
+}
+
+// First index of CTA c's list when U ranks are dealt in zigzag rounds of C.
+__host__ __device__ __forceinline__ long long zigzag_start(long long c, long long U, long long C)
+{
+    const long long full = U / C, R = U % C;
+    long long extra = 0;
+    if (R) extra = (full & 1) ? ((c > C - R) ? c - (C - R) : 0) : (c < R ? c : R);
+    return c * full + extra;
+}
+
+__global__ void __launch_bounds__(1024) sched_assign_kernel(Geo g, int C, const int32_t *__restrict__ unit_cost,
+                                                            const int32_t *__restrict__ head_sorted,
+                                                            const int64_t *__restrict__ head_cost,
+                                                            int32_t *__restrict__ work, int32_t *__restrict__ cta_range,
+                                                            int64_t *__restrict__ cta_cost, int hpow2)
+{
+    extern __shared__ unsigned long long sa_smem[];
+    unsigned long long *hkeys = sa_smem;          // [hpow2]
+    unsigned long long *ccost = sa_smem + hpow2;  // [C]
+    for (int h = threadIdx.x; h < hpow2; h += blockDim.x) {
+        if (h < g.BH) {
+            const unsigned long long c = (unsigned long long)head_cost[h];
+            hkeys[h] = ((0xFFFFFFFFull - (c & 0xFFFFFFFFull)) << 32) | (uint32_t)h;
+        } else {
+            hkeys[h] = ~0ull;
+        }
+    }
+    for (int c = threadIdx.x; c < C; c += blockDim.x) ccost[c] = 0ull;
+    __syncthreads();
+    bitonic_sort_u64(hkeys, hpow2);
+    const long long U = (long long)g.BH * g.nb;
+    for (int c = threadIdx.x; c <= C; c += blockDim.x) cta_range[c] = (int32_t)zigzag_start(c, U, C);
+    for (long long r = threadIdx.x; r < U; r += blockDim.x) {
+        const long long hr = r / g.nb, local = r - hr * g.nb;
+        const int head = (int)(hkeys[hr] & 0xFFFFFFFFull);
+        const int i = head_sorted[(size_t)head * g.nb + local];
+        const long long u = (long long)head * g.nb + i;
+        const long long round = r / C, pos = r - round * C;
+        const long long c = (round & 1) ? (C - 1 - pos) : pos;
+        work[zigzag_start(c, U, C) + round] = (int32_t)u;
+        atomicAdd(&ccost[c], (unsigned long long)unit_cost[u]);
+    }
+    __syncthreads();
+    if (cta_cost)
+        for (int c = threadIdx.x; c < C; c += blockDim.x) cta_cost[c] = (int64_t)ccost[c];
+}
+
+static int next_pow2(int n)
+{
+    int p = 1;
+    while (p < n) p <<= 1;
+    return p;
+}
+
+cudaError_t launch_schedule(const Geo &g, const int32_t *kv_cnt, const int32_t *kv_idx, int dense, int num_ctas,
+                            int32_t *work, int32_t *cta_range, int64_t *cta_cost, int32_t *unit_cost,
+                            int32_t *head_sorted, int64_t *head_cost, cudaStream_t stream)
+{
+    const int npow2 = next_pow2(g.nb);
+    const size_t smem_a = (size_t)npow2 * sizeof(unsigned long long);
+    cudaError_t err = cudaFuncSetAttribute(sched_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a);
+    if (err != cudaSuccess) return err;
+    sched_head_kernel<<<g.BH, 1024, smem_a, stream>>>(g, kv_cnt, kv_idx, dense, unit_cost, head_sorted, head_cost,
+                                                      npow2);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    const int hpow2 = next_pow2(g.BH);
+    const size_t smem_b = ((size_t)hpow2 + num_ctas) * sizeof(unsigned long long);
+    err = cudaFuncSetAttribute(sched_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b);
+    if (err != cudaSuccess) return err;
+    sched_assign_kernel<<<1, 1024, smem_b, stream>>>(g, num_ctas, unit_cost, head_sorted, head_cost, work,
+                                                     cta_range, cta_cost, hpow2);
+    return cudaGetLastError();
+}
+
+}  // namespace fvattn

@@ -1,0 +1,234 @@
+"""Thin ctypes binding of the C-ABI library `libfvattn.so` (include/fvattn.h).
+
+Every function here only checks and marshals arguments (torch tensors ->
+device pointers, the current CUDA stream) and calls the library; all
+computation runs in the library's CUDA kernels. Importing this module loads
+the library and raises if it is missing: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfvattn.so")
+
+OK, INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA_ERR, NONFINITE, TIMEOUT = range(7)
+FLAG_NONFINITE, FLAG_TIMEOUT = 0x1, 0x2
+
+
+class FVAttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "N", "D", "grid_t", "grid_h", "grid_w",
+                                              "blk_t", "blk_h", "blk_w")] + [("softmax_scale", ctypes.c_float)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing; build it with "
+                          "`python -m block_sparse_attention_fvattn_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    P = ctypes.POINTER(Problem)
+    sig = {
+        "fvattn_num_blocks": (i32, [P]),
+        "fvattn_default_num_ctas": (i32, []),
+        "fvattn_workspace_size": (sz, [P, i32]),
+        "fvattn_workspace_init": (i32, [vp, sz, vp]),
+        "fvattn_route": (i32, [P, vp, vp, f32, i32, vp, vp, vp, vp, sz, vp]),
+        "fvattn_schedule": (i32, [P, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp]),
+        "fvattn_sparse_attn": (i32, [P, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]),
+        "fvattn_read_device_status": (i32, [vp, vp, ctypes.POINTER(ctypes.c_uint32)]),
+        "fvattn_status_string": (ctypes.c_char_p, [i32]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+_lib = _load()
+EXPORTED = ("fvattn_num_blocks", "fvattn_default_num_ctas", "fvattn_workspace_size", "fvattn_workspace_init",
+            "fvattn_route", "fvattn_schedule", "fvattn_sparse_attn", "fvattn_read_device_status",
+            "fvattn_status_string")
+
+
+def status_string(s: int) -> str:
+    return _lib.fvattn_status_string(int(s)).decode()
+
+
+@dataclass(frozen=True)
+class Geometry:
+    B: int
+    H: int
+    D: int
+    grid: Tuple[int, int, int]
+    block: Tuple[int, int, int]
+    softmax_scale: float = 0.0   # <= 0 selects 1/sqrt(D)
+
+    @property
+    def N(self) -> int:
+        return self.grid[0] * self.grid[1] * self.grid[2]
+
+    def problem(self) -> Problem:
+        T, Hg, W = self.grid
+        bt, bh, bw = self.block
+        return Problem(self.B, self.H, self.N, self.D, T, Hg, W, bt, bh, bw, float(self.softmax_scale))
+
+    @property
+    def scale(self) -> float:
+        return self.softmax_scale if self.softmax_scale > 0 else 1.0 / math.sqrt(self.D)
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _check(st: int, where: str):
+    if st != OK:
+        raise FVAttnError(st, where)
+
+
+def num_blocks(geo: Geometry) -> int:
+    p = geo.problem()
+    return int(_lib.fvattn_num_blocks(ctypes.byref(p)))
+
+
+def default_num_ctas() -> int:
+    return int(_lib.fvattn_default_num_ctas())
+
+
+def workspace_size(geo: Geometry, num_ctas: int = 0) -> int:
+    p = geo.problem()
+    return int(_lib.fvattn_workspace_size(ctypes.byref(p), int(num_ctas)))
+
+
+def workspace_init(ws: torch.Tensor, stream=None):
+    _check(_lib.fvattn_workspace_init(_ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)),
+           "fvattn_workspace_init")
+
+
+def route(geo: Geometry, q: torch.Tensor, k: torch.Tensor, p: float, k_min: int,
+          kv_cnt: torch.Tensor, kv_idx: torch.Tensor, ws: torch.Tensor,
+          block_probs: Optional[torch.Tensor] = None, stream=None):
+    prob = geo.problem()
+    st = _lib.fvattn_route(ctypes.byref(prob), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+                           float(p), int(k_min), _ptr(kv_cnt, torch.int32, "kv_cnt"),
+                           _ptr(kv_idx, torch.int32, "kv_idx"), _ptr(block_probs, torch.float32, "block_probs"),
+                           _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check(st, "fvattn_route")
+
+
+def schedule(geo: Geometry, kv_cnt: Optional[torch.Tensor], kv_idx: Optional[torch.Tensor], dense: bool,
+             num_ctas: int, work: torch.Tensor, cta_range: torch.Tensor, ws: torch.Tensor,
+             cta_cost: Optional[torch.Tensor] = None, stream=None):
+    prob = geo.problem()
+    st = _lib.fvattn_schedule(ctypes.byref(prob), _ptr(kv_cnt, torch.int32, "kv_cnt"),
+                              _ptr(kv_idx, torch.int32, "kv_idx"), int(bool(dense)), int(num_ctas),
+                              _ptr(work, torch.int32, "work"), _ptr(cta_range, torch.int32, "cta_range"),
+                              _ptr(cta_cost, torch.int64, "cta_cost"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+                              _stream(stream))
+    _check(st, "fvattn_schedule")
+
+
+def sparse_attn(geo: Geometry, q, k, v, kv_cnt, kv_idx, work, cta_range, num_ctas: int, dense: bool,
+                out: torch.Tensor, ws: torch.Tensor, cta_ns: Optional[torch.Tensor] = None, stream=None):
+    prob = geo.problem()
+    st = _lib.fvattn_sparse_attn(ctypes.byref(prob), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+                                 _ptr(v, torch.bfloat16, "v"), _ptr(kv_cnt, torch.int32, "kv_cnt"),
+                                 _ptr(kv_idx, torch.int32, "kv_idx"), _ptr(work, torch.int32, "work"),
+                                 _ptr(cta_range, torch.int32, "cta_range"), int(num_ctas), int(bool(dense)),
+                                 _ptr(out, torch.bfloat16, "out"), _ptr(cta_ns, torch.int64, "cta_ns"),
+                                 _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check(st, "fvattn_sparse_attn")
+
+
+def read_device_status(ws: torch.Tensor, stream=None) -> int:
+    flags = ctypes.c_uint32(0)
+    _check(_lib.fvattn_read_device_status(_ptr(ws, torch.uint8, "ws"), _stream(stream), ctypes.byref(flags)),
+           "fvattn_read_device_status")
+    return int(flags.value)
+
+
+class FVAttn:
+    """The whole path for one problem: route -> schedule -> block-sparse attention.
+
+    Buffers (lists, schedule, workspace) are allocated once through torch and
+    reused; `__call__` enqueues the three library calls on the current stream.
+    """
+
+    def __init__(self, geo: Geometry, p: float, k_min: int, device="cuda", num_ctas: int = 0,
+                 with_probs: bool = False):
+        self.geo, self.p, self.k_min = geo, float(p), int(k_min)
+        self.nb = num_blocks(geo)
+        if self.nb < 0:
+            raise FVAttnError(INVALID_ARG, "FVAttn")
+        self.num_ctas = num_ctas if num_ctas > 0 else default_num_ctas()
+        dev = torch.device(device)
+        B, H, nb = geo.B, geo.H, self.nb
+        self.kv_cnt = torch.zeros((B, H, nb), dtype=torch.int32, device=dev)
+        self.kv_idx = torch.zeros((B, H, nb, nb), dtype=torch.int32, device=dev)
+        self.block_probs = torch.zeros((B, H, nb, nb), dtype=torch.float32, device=dev) if with_probs else None
+        self.work = torch.zeros(B * H * nb, dtype=torch.int32, device=dev)
+        self.cta_range = torch.zeros(self.num_ctas + 1, dtype=torch.int32, device=dev)
+        self.cta_cost = torch.zeros(self.num_ctas, dtype=torch.int64, device=dev)
+        self.cta_ns = torch.zeros(self.num_ctas, dtype=torch.int64, device=dev)
+        self.dense_work = torch.zeros_like(self.work)
+        self.dense_range = torch.zeros_like(self.cta_range)
+        self.ws = torch.zeros(max(workspace_size(geo, self.num_ctas), 256), dtype=torch.uint8, device=dev)
+        workspace_init(self.ws)
+        self._dense_scheduled = False
+
+    def route(self, q, k, stream=None):
+        route(self.geo, q, k, self.p, self.k_min, self.kv_cnt, self.kv_idx, self.ws, self.block_probs, stream)
+
+    def schedule(self, stream=None):
+        schedule(self.geo, self.kv_cnt, self.kv_idx, False, self.num_ctas, self.work, self.cta_range, self.ws,
+                 self.cta_cost, stream)
+
+    def attend(self, q, k, v, out, stream=None, timing=False):
+        sparse_attn(self.geo, q, k, v, self.kv_cnt, self.kv_idx, self.work, self.cta_range, self.num_ctas,
+                    False, out, self.ws, self.cta_ns if timing else None, stream)
+
+    def dense(self, q, k, v, out, stream=None, timing=False):
+        if not self._dense_scheduled:
+            schedule(self.geo, None, None, True, self.num_ctas, self.dense_work, self.dense_range, self.ws,
+                     None, stream)
+            self._dense_scheduled = True
+        sparse_attn(self.geo, q, k, v, None, None, self.dense_work, self.dense_range, self.num_ctas, True, out,
+                    self.ws, self.cta_ns if timing else None, stream)
+
+    def __call__(self, q, k, v, out=None, stream=None):
+        if out is None:
+            out = torch.empty_like(q)
+        self.route(q, k, stream)
+        self.schedule(stream)
+        self.attend(q, k, v, out, stream)
+        return out
+
+    def status(self, stream=None) -> int:
+        return read_device_status(self.ws, stream)

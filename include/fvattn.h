@@ -1,0 +1,198 @@
+/*
+ * fvattn.h -- C ABI of the B200 (sm_100a) adaptive block-sparse attention path.
+ *
+ * The method (FVAttn, "Adaptive Sparse Attention with Runtime Load Balancing
+ * for Video Generation"; ai-feeds.com summary and hotpaper.ai abstract) routes
+ * each query block of a video DiT's self-attention to a Top-p set of key/value
+ * blocks with a Top-k safety floor over video-aware spatio-temporal blocks,
+ * repairs the mask, balances the resulting uneven per-head work, and runs
+ * attention only over the kept blocks. This library implements the
+ * single-GPU data path of that method in three calls:
+ *
+ *   fvattn_route        block pooling, block scores, softmax, Top-p + Top-k
+ *                       floor, mask repair, compact per-(head, query block)
+ *                       key/value block lists
+ *   fvattn_schedule     longest-first, balanced work lists for persistent CTAs
+ *   fvattn_sparse_attn  FlashAttention-style online-softmax attention over the
+ *                       kept blocks only (or every block: dense mode)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Tensors.  Q, K, V and O are bf16, contiguous, [B, H, N, D] (row-major, D
+ *   innermost). Token n of a head sits at latent position (t, y, x) with
+ *   n = (t * grid_h + y) * grid_w + x (raster order, T slowest), as in the
+ *   FastVideo VSA backend's (T, H, W) post-patch latent grid (zskr.cn guide,
+ *   section 1). Q and KV have the same length (non-causal self-attention,
+ *   zskr.cn guide, section 1) and the same head count (no GQA/MQA, section 5).
+ * Blocks.  The grid is cut into (blk_t, blk_h, blk_w) blocks; the block count
+ *   is nb = ceil(T/bt) * ceil(H/bh) * ceil(W/bw) (zskr.cn guide, section 3:
+ *   (31,22,40) with (4,8,8) gives 8*3*5 = 120). Block j = (jt*nbh + jy)*nbw + jx.
+ *   Edge blocks hold fewer valid tokens; padded positions never act as keys
+ *   and never produce output (section 6, packed [real, pad] contract).
+ *   Supported: blk_t*blk_h*blk_w == 256 with blk_t even (the 256-token route,
+ *   e.g. (4,8,8)) or == 64 (the 64-token (4,4,4) route, section 1), blk_w and
+ *   blk_h <= 256; D in {64, 128}; nb <= 2048; B*H <= 65535.
+ * Pointers.  Device pointers unless stated; 16-byte aligned. The caller owns
+ *   every buffer. The library allocates no device memory; the only state it
+ *   keeps is per-device function attributes and a cached driver entry point.
+ * Streams.  Every call is asynchronous on `stream` (a cudaStream_t; NULL is
+ *   the legacy default stream). Argument errors are returned synchronously,
+ *   before anything is enqueued. No call synchronises with the host except
+ *   fvattn_read_device_status.
+ * Workspace.  One caller-owned device buffer of fvattn_workspace_size() bytes
+ *   serves all three calls of one problem; fvattn_workspace_init must run on
+ *   it once before first use. It holds the sticky device status word, the
+ *   pooled block means and the scheduler's scratch. Calls that share a
+ *   workspace must be ordered on one stream.
+ * Device-detected conditions (non-finite block scores, a bounded wait that
+ *   ran out) never trap: kernels OR a flag into the workspace status word,
+ *   which fvattn_read_device_status returns.
+ */
+#ifndef FVATTN_H
+#define FVATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FVATTN_API __attribute__((visibility("default")))
+#else
+#define FVATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so this header needs no CUDA header. */
+typedef struct CUstream_st *fvattn_stream_t;
+
+typedef enum fvattn_status {
+    FVATTN_OK = 0,
+    FVATTN_ERR_INVALID_ARG = 1,   /* a size, pointer, p or k_min out of range */
+    FVATTN_ERR_UNSUPPORTED = 2,   /* valid problem outside the supported shapes */
+    FVATTN_ERR_WORKSPACE = 3,     /* workspace NULL or smaller than required */
+    FVATTN_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed */
+    FVATTN_STATUS_NONFINITE = 5,  /* device flag: a score row was not finite and was repaired */
+    FVATTN_ERR_TIMEOUT = 6        /* device flag: a bounded wait inside a kernel gave up */
+} fvattn_status;
+
+/* Device status word bits (as returned, combined, by fvattn_read_device_status). */
+#define FVATTN_FLAG_NONFINITE 0x1u
+#define FVATTN_FLAG_TIMEOUT 0x2u
+
+typedef struct fvattn_problem {
+    int32_t B, H, N, D;               /* batch, heads, tokens (= T*Hg*W), head dim */
+    int32_t grid_t, grid_h, grid_w;   /* latent grid (T, H, W) */
+    int32_t blk_t, blk_h, blk_w;      /* block shape */
+    float softmax_scale;              /* <= 0 selects 1/sqrt(D); used for routing and attention */
+} fvattn_problem;
+
+/* nb = ceil(T/bt)*ceil(H/bh)*ceil(W/bw), or -1 if the problem is invalid. */
+FVATTN_API int32_t fvattn_num_blocks(const fvattn_problem *prob);
+
+/* Number of SMs of the current device (the default persistent-CTA count), or -1. */
+FVATTN_API int32_t fvattn_default_num_ctas(void);
+
+/* Bytes of workspace the three calls need for `prob` with `num_ctas` persistent
+ * CTAs (0 = fvattn_default_num_ctas()). Returns 0 if the problem is invalid. */
+FVATTN_API size_t fvattn_workspace_size(const fvattn_problem *prob, int32_t num_ctas);
+
+/* Zero the workspace header (status word and counters). Asynchronous. */
+FVATTN_API fvattn_status fvattn_workspace_init(void *ws, size_t ws_bytes, fvattn_stream_t stream);
+
+/*
+ * fvattn_route -- the sparse-routing frontend (ai-feeds.com FVAttn summary,
+ * "Key modules" 1: Top-p routing with a Top-k safety floor over video-aware
+ * blocks, runtime mask repair; hotpaper.ai abstract; zskr.cn guide, section 1:
+ * block-level scores select key/value blocks per query block).
+ *
+ * For every (b, h, query block i):
+ *   Qbar_i, Kbar_j = means of Q, K over the valid tokens of the block;
+ *   s[j] = scale * dot(Qbar_i, Kbar_j);  P = softmax(s);
+ *   rank blocks by P descending (= s descending), equal scores by lower j;
+ *   m_p = smallest m whose inclusive cumulative P reaches p (p >= 1: nb);
+ *   m = min(nb, max(m_p, k_min)); S_i = first m ranked blocks plus block i;
+ *   a row with a non-finite score keeps every block and sets FLAG_NONFINITE.
+ *
+ *   q, k          bf16 [B,H,N,D]
+ *   p             Top-p threshold, 0 < p <= 1
+ *   k_min         Top-k floor, 1 <= k_min <= nb (k_min > nb is INVALID_ARG,
+ *                 k_min == nb keeps every block, like VSA's topk rules,
+ *                 zskr.cn guide, section 3)
+ *   kv_cnt        out int32 [B,H,nb]      |S_i|
+ *   kv_idx        out int32 [B,H,nb,nb]   S_i ascending in the first kv_cnt
+ *                 entries of each row; the rest of the row is left untouched
+ *   block_probs   out fp32 [B,H,nb,nb] P in block order, or NULL
+ *   ws, ws_bytes  workspace
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE (synchronous); CUDA on a failed
+ * launch.
+ */
+FVATTN_API fvattn_status fvattn_route(const fvattn_problem *prob, const void *q, const void *k,
+                           float p, int32_t k_min, int32_t *kv_cnt, int32_t *kv_idx,
+                           float *block_probs, void *ws, size_t ws_bytes, fvattn_stream_t stream);
+
+/*
+ * fvattn_schedule -- longest-first balanced work lists for the persistent
+ * attention CTAs: the single-GPU analogue of the method's per-head load
+ * problem (ai-feeds.com summary: per-head workload heterogeneity makes the
+ * heaviest rank the critical path; Runtime Load Balancing moves heavy heads
+ * to shorten it; load imbalance = max/mean, ideal 1.0).
+ *
+ * A work unit is one (b, h, query block i). Its cost is the number of
+ * (128-row query tile, key/value sub-tile) pairs the attention kernel runs for
+ * it. Units are ordered heads by total cost descending, then units within a
+ * head by cost descending (ties: lower index); rank r goes to CTA
+ * zigzag(r) = r mod 2C < C ? r mod C : 2C-1 - r mod C, so each round of C
+ * consecutive ranks (one head's units run together, which keeps its key/value
+ * blocks in L2) gives every CTA one unit, alternating the largest end.
+ *
+ *   kv_cnt, kv_idx  the lists from fvattn_route (ignored if dense != 0)
+ *   dense           nonzero: schedule the all-blocks problem
+ *   num_ctas        persistent CTAs (0 = SM count)
+ *   work            out int32 [B*H*nb]    unit ids u = (b*H + h)*nb + i, grouped by CTA
+ *   cta_range       out int32 [num_ctas+1] CTA c runs work[cta_range[c] .. cta_range[c+1])
+ *   cta_cost        out int64 [num_ctas]  predicted cost per CTA, or NULL
+ */
+FVATTN_API fvattn_status fvattn_schedule(const fvattn_problem *prob, const int32_t *kv_cnt,
+                              const int32_t *kv_idx, int32_t dense, int32_t num_ctas,
+                              int32_t *work, int32_t *cta_range, int64_t *cta_cost,
+                              void *ws, size_t ws_bytes, fvattn_stream_t stream);
+
+/*
+ * fvattn_sparse_attn -- block-sparse attention over the kept blocks (the
+ * source of the method's 4.41x attention speedup over FlashAttention,
+ * ai-feeds.com summary "Key findings"; zskr.cn guide, section 1: attention is
+ * computed only for the selected key/value blocks of each query block).
+ *
+ * For every valid query token r of block i: o_r = sum over the valid tokens k
+ * of the blocks in S_i of softmax_k(scale * q_r . k_k) * v_k, computed with an
+ * online softmax over 128-token (64 for 64-token blocks) key/value sub-tiles.
+ * dense != 0 uses every block (the VSA_ALL_BLOCKS route, section 3/5), giving
+ * the in-library dense comparison.
+ *
+ *   q, k, v        bf16 [B,H,N,D]
+ *   kv_cnt, kv_idx lists from fvattn_route (ignored if dense)
+ *   work, cta_range from fvattn_schedule with the same num_ctas and dense flag
+ *   num_ctas       grid size (0 = SM count); must match fvattn_schedule's
+ *   out            bf16 [B,H,N,D]; every valid token is written
+ *   cta_ns         out int64 [num_ctas] busy time of each CTA in ns, or NULL
+ */
+FVATTN_API fvattn_status fvattn_sparse_attn(const fvattn_problem *prob, const void *q, const void *k,
+                                 const void *v, const int32_t *kv_cnt, const int32_t *kv_idx,
+                                 const int32_t *work, const int32_t *cta_range, int32_t num_ctas,
+                                 int32_t dense, void *out, int64_t *cta_ns,
+                                 void *ws, size_t ws_bytes, fvattn_stream_t stream);
+
+/* Synchronise `stream`, return the device status word's flags (FVATTN_FLAG_*)
+ * in *flags, and clear them. Returns CUDA on a failed copy. */
+FVATTN_API fvattn_status fvattn_read_device_status(void *ws, fvattn_stream_t stream, uint32_t *flags);
+
+/* Static description of a status code. */
+FVATTN_API const char *fvattn_status_string(fvattn_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FVATTN_H */

@@ -1,0 +1,127 @@
+"""Edge cases and special cases of the CUDA path (needs a B200)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_fvattn_b200 import inputs as gen
+from tests import fvtest
+
+pytestmark = pytest.mark.gpu
+
+
+def _engine(wl, **kw):
+    from block_sparse_attention_fvattn_b200 import fvattn as fa
+    return fa.FVAttn(fvtest.geometry(wl), wl.p, wl.k_min, **kw)
+
+
+def test_floor_equal_to_num_blocks_is_dense():
+    # VSA accepts topk == num_blocks (zskr.cn guide, section 3): every block is kept,
+    # and the sparse kernel then reproduces dense mode exactly (same tiles, same order)
+    wl0 = gen.custom("kmin_nb", 1, 2, 128, (9, 20, 28), (4, 8, 8), 0.5, 1, sigma=2.0, a_range=(0.5, 4.0), seed=31)
+    from block_sparse_attention_fvattn_b200 import fvattn as fa
+    nb = fa.num_blocks(fvtest.geometry(wl0))
+    wl = gen.custom("kmin_nb", 1, 2, 128, (9, 20, 28), (4, 8, 8), 0.5, nb, sigma=2.0, a_range=(0.5, 4.0), seed=31)
+    q, k, v = fvtest.make_on_gpu(wl)
+    eng = _engine(wl)
+    out = eng(q, k, v)
+    assert (eng.kv_cnt == nb).all()
+    assert (eng.kv_idx == torch.arange(nb, device="cuda", dtype=torch.int32)).all()
+    dense = torch.empty_like(q)
+    eng.dense(q, k, v, dense)
+    torch.cuda.synchronize()
+    assert torch.equal(out, dense)
+
+
+def test_p_one_keeps_every_block():
+    wl = gen.custom("p1", 1, 2, 64, (8, 16, 24), (4, 8, 8), 1.0, 1, sigma=2.0, a_range=(2.0, 4.0), seed=32)
+    q, k, v = fvtest.make_on_gpu(wl)
+    eng = _engine(wl)
+    eng.route(q, k)
+    torch.cuda.synchronize()
+    assert (eng.kv_cnt == eng.nb).all()
+
+
+def test_tiny_p_is_top1_plus_diagonal():
+    wl = gen.custom("p_tiny", 1, 2, 128, (12, 24, 24), (4, 8, 8), 1e-6, 1, sigma=2.0, a_range=(0.5, 4.0), seed=33)
+    q, k, v = fvtest.make_on_gpu(wl)
+    eng = _engine(wl)
+    eng.route(q, k)
+    torch.cuda.synchronize()
+    cnt = eng.kv_cnt.cpu().numpy()
+    assert ((cnt == 1) | (cnt == 2)).all()
+
+
+def test_grid_smaller_than_one_block():
+    # Sol-Attn's "seq_len < block_size" case (bjdmk.com.cn, section 6.1): one partial block
+    import oracle
+    wl = gen.custom("sub_block", 1, 3, 128, (2, 3, 5), (4, 8, 8), 0.9, 1, sigma=1.0, a_range=(0.5, 4.0), seed=34)
+    q, k, v = fvtest.make_on_gpu(wl)
+    eng = _engine(wl)
+    out = eng(q, k, v)
+    torch.cuda.synchronize()
+    assert eng.nb == 1 and (eng.kv_cnt == 1).all()
+    orc = oracle.get()
+    g = orc.geom(1, 3, wl.grid, wl.block, 128)
+    rows = np.arange(3 * wl.N)
+    ref, _ = orc.attn_rows(g, q.cpu(), k.cpu(), v.cpu(), 1 / math.sqrt(128), rows)
+    mx, mean = fvtest.attn_errors(out, rows, ref, 128)
+    assert mx <= fvtest.ATTN_MAX_ABS and mean <= fvtest.ATTN_MEAN_ABS
+
+
+def test_nonfinite_scores_are_repaired_and_flagged():
+    from block_sparse_attention_fvattn_b200 import fvattn as fa
+    wl = gen.custom("nonfinite", 1, 2, 128, (8, 16, 16), (4, 8, 8), 0.5, 1, sigma=2.0, a_range=(1.0, 4.0), seed=35)
+    q, k, v = fvtest.make_on_gpu(wl)
+    q[0, 1, 5] = float("inf")          # token 5 lies in block 0 of head 1
+    eng = _engine(wl)
+    eng.route(q, k)
+    flags = eng.status()
+    assert flags & fa.FLAG_NONFINITE
+    assert int(eng.kv_cnt[0, 1, 0]) == eng.nb
+    assert eng.status() == 0           # reading clears the flag
+
+
+def test_empty_batch_is_a_no_op():
+    from block_sparse_attention_fvattn_b200 import fvattn as fa
+    geo = fa.Geometry(0, 4, 128, (8, 16, 16), (4, 8, 8))
+    ws = torch.zeros(max(fa.workspace_size(geo), 256), dtype=torch.uint8, device="cuda")
+    fa.workspace_init(ws)
+    e = torch.empty((0, 4, 2048, 128), dtype=torch.bfloat16, device="cuda")
+    cnt = torch.empty((0,), dtype=torch.int32, device="cuda")
+    # zero-element tensors have no storage; pass any aligned allocation
+    buf = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
+    ibuf = torch.zeros(16, dtype=torch.int32, device="cuda")
+    fa.route(geo, buf, buf, 0.9, 1, ibuf, ibuf, ws)
+    work = torch.zeros(4, dtype=torch.int32, device="cuda")
+    rng = torch.zeros(9, dtype=torch.int32, device="cuda")
+    fa.schedule(geo, ibuf, ibuf, False, 8, work, rng, ws)
+    fa.sparse_attn(geo, buf, buf, buf, ibuf, ibuf, work, rng, 8, False, buf, ws)
+    torch.cuda.synchronize()
+    assert (rng == 0).all()
+    del e, cnt
+
+
+@pytest.mark.parametrize("num_ctas", [1, 7, 148, 300])
+def test_output_independent_of_cta_count(num_ctas):
+    wl = gen.custom("ctas", 1, 3, 128, (9, 20, 28), (4, 8, 8), 0.9, 4, sigma=2.0, a_range=(0.5, 4.0), seed=36)
+    q, k, v = fvtest.make_on_gpu(wl)
+    ref = _engine(wl, num_ctas=148)(q, k, v)
+    out = _engine(wl, num_ctas=num_ctas)(q, k, v)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+
+
+def test_repeatable():
+    wl = gen.WORKLOADS["wan5b"]
+    q, k, v = fvtest.make_on_gpu(wl)
+    eng = _engine(wl)
+    o1 = eng(q, k, v).clone()
+    c1, i1 = eng.kv_cnt.clone(), eng.kv_idx.clone()
+    o2 = eng(q, k, v)
+    torch.cuda.synchronize()
+    assert torch.equal(c1, eng.kv_cnt)
+    assert torch.equal(o1, o2)
+    mask = torch.arange(eng.nb, device="cuda")[None, None, None, :] < c1[..., None]
+    assert torch.equal(torch.where(mask, i1, 0), torch.where(mask, eng.kv_idx, 0))

@@ -1,0 +1,148 @@
+"""CUDA path vs the fp64 oracle, through the C ABI (needs a B200).
+
+Per workload: routing lists (bit-exact except the stated boundary excuses)
+and block probabilities, the schedule (exact, recomputed on the host), and
+attention on the GPU's own lists against the oracle -- every query row for
+the small ragged cases, sampled rows (edges, heaviest and lightest units,
+random) for the five full-size workloads, in the launch configuration the
+benchmark uses (one persistent CTA per SM, scheduled work lists).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_fvattn_b200 import inputs as gen
+from tests import fvtest
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    gen.custom("ragged_256tok", 1, 3, 128, (9, 20, 28), (4, 8, 8), 0.9, 4, sigma=2.0, a_range=(0.5, 4.0), seed=21),
+    gen.custom("last_frame_only", 1, 2, 128, (5, 11, 13), (4, 8, 8), 0.8, 2, sigma=1.5, a_range=(0.5, 4.0),
+               seed=22),
+    gen.custom("d64_b2", 2, 2, 64, (8, 16, 24), (4, 8, 8), 0.9, 2, sigma=2.0, a_range=(0.5, 3.0), seed=23),
+    gen.custom("blk64", 1, 4, 128, (8, 12, 20), (4, 4, 4), 0.95, 4, sigma=2.0, a_range=(0.25, 6.0), seed=24),
+    gen.custom("blk64_ragged_d64", 1, 2, 64, (6, 10, 9), (4, 4, 4), 0.9, 3, sigma=1.5, a_range=(0.5, 4.0),
+               seed=25),
+    gen.custom("iid_tiny", 1, 2, 64, (8, 16, 16), (4, 8, 8), 0.9, 2, seed=26),
+]
+FULL = [gen.WORKLOADS[n] for n in gen.WORKLOAD_ORDER]
+
+
+def _oracle_route(orc, wl, q, k):
+    g = orc.geom(wl.B, wl.H, wl.grid, wl.block, wl.D)
+    qb, kb = orc.pool(g, q), orc.pool(g, k)
+    r = orc.route(g, qb, kb, 1.0 / math.sqrt(wl.D), wl.p, wl.k_min)
+    return g, qb, kb, r
+
+
+def _host_costs(wl, nb, kv_cnt, kv_idx):
+    """Cost of every unit as the scheduler defines it, recomputed on the host:
+    active 128-row query tiles x kept key/value sub-tiles."""
+    T, Hg, W = wl.grid
+    bt, bh, bw = wl.block
+    nbh, nbw = -(-Hg // bh), -(-W // bw)
+    two = bt * bh * bw == 256
+    subt = bt // 2 if two else bt
+
+    def nsub(j):
+        jt = j // (nbh * nbw)
+        return 1 + (1 if two and jt * bt + subt < T else 0)
+
+    ns = np.array([nsub(j) for j in range(nb)])
+    nh = np.array([1 + (1 if two and (i // (nbh * nbw)) * bt + subt < T else 0) for i in range(nb)])
+    BH = wl.B * wl.H
+    cnt = kv_cnt.reshape(BH, nb)
+    idx = kv_idx.reshape(BH, nb, nb)
+    cost = np.zeros((BH, nb), dtype=np.int64)
+    for h in range(BH):
+        for i in range(nb):
+            cost[h, i] = nh[i] * ns[idx[h, i, :cnt[h, i]]].sum()
+    return cost
+
+
+def _expected_work(cost, C):
+    BH, nb = cost.shape
+    heads = sorted(range(BH), key=lambda h: (-cost[h].sum(), h))
+    ranked = []
+    for h in heads:
+        ranked += [h * nb + i for i in sorted(range(nb), key=lambda i: (-cost[h, i], i))]
+    lists = [[] for _ in range(C)]
+    for r, u in enumerate(ranked):
+        rd, pos = divmod(r, C)
+        lists[C - 1 - pos if rd % 2 else pos].append(u)
+    return lists
+
+
+def _run(wl, full_rows):
+    import oracle
+    from block_sparse_attention_fvattn_b200 import fvattn as fa
+    orc = oracle.get()
+    q, k, v = fvtest.make_on_gpu(wl)
+    geo = fvtest.geometry(wl)
+    eng = fa.FVAttn(geo, wl.p, wl.k_min, with_probs=True)
+    eng.route(q, k)
+    eng.schedule()
+    out = torch.zeros_like(q)
+    eng.attend(q, k, v, out, timing=True)
+    out_dense = torch.zeros_like(q)
+    eng.dense(q, k, v, out_dense)
+    torch.cuda.synchronize()
+    assert eng.status() == 0
+    qh, kh, vh = q.cpu(), k.cpu(), v.cpu()
+    g, qb, kb, r = _oracle_route(orc, wl, qh, kh)
+    nb = eng.nb
+    cnt = eng.kv_cnt.cpu().numpy()
+    idx = eng.kv_idx.cpu().numpy()
+
+    # ---- routing
+    cmp = fvtest.compare_lists(cnt, idx, r, qb, kb, geo.scale, wl.p, wl.k_min)
+    assert cmp.unexcused == 0, cmp
+    assert cmp.excused_topp + cmp.excused_tie <= max(2, 0.02 * cmp.rows), cmp
+    probs = eng.block_probs.cpu().numpy().astype(np.float64)
+    np.testing.assert_allclose(probs, r["probs"], rtol=2e-3, atol=1e-6)
+    # invariants of the GPU's own lists
+    for_rows = cnt.reshape(-1)
+    assert (for_rows >= min(wl.k_min, nb)).all() and (for_rows <= nb).all()
+
+    # ---- schedule
+    C = eng.num_ctas
+    work = eng.work.cpu().numpy()
+    rng = eng.cta_range.cpu().numpy()
+    U = wl.B * wl.H * nb
+    assert rng[0] == 0 and rng[C] == U and (np.diff(rng) >= 0).all()
+    assert np.array_equal(np.sort(work), np.arange(U))
+    cost = _host_costs(wl, nb, cnt, idx)
+    expect = _expected_work(cost, C)
+    for c in range(C):
+        assert work[rng[c]:rng[c + 1]].tolist() == expect[c], c
+    cta_cost = eng.cta_cost.cpu().numpy()
+    flat = cost.reshape(-1)
+    assert all(cta_cost[c] == flat[work[rng[c]:rng[c + 1]]].sum() for c in range(C))
+    ns = eng.cta_ns.cpu().numpy()
+    assert (ns[np.diff(rng) > 0] > 0).all()
+
+    # ---- attention on the GPU's own lists, and dense mode
+    rows = np.arange(wl.B * wl.H * wl.N) if full_rows else fvtest.sample_rows(wl, cnt)
+    ref, wsum = orc.attn_rows(g, qh, kh, vh, geo.scale, rows, cnt, idx)
+    assert np.abs(wsum - 1.0).max() < 1e-9
+    mx, mean = fvtest.attn_errors(out, rows, ref, wl.D)
+    assert mx <= fvtest.ATTN_MAX_ABS and mean <= fvtest.ATTN_MEAN_ABS, (mx, mean)
+    assert torch.isfinite(out).all()
+    drows = rows if full_rows else rows[:: max(1, len(rows) // 48)]
+    dref, _ = orc.attn_rows(g, qh, kh, vh, geo.scale, drows)
+    dmx, dmean = fvtest.attn_errors(out_dense, drows, dref, wl.D)
+    assert dmx <= fvtest.ATTN_MAX_ABS and dmean <= fvtest.ATTN_MEAN_ABS, (dmx, dmean)
+    return dict(cmp=cmp, max_abs=mx, mean_abs=mean, dense_max=dmx)
+
+
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
+def test_small_every_row(wl):
+    _run(wl, full_rows=True)
+
+
+@pytest.mark.parametrize("wl", FULL, ids=lambda w: w.name)
+def test_full_size_sampled(wl):
+    _run(wl, full_rows=False)
