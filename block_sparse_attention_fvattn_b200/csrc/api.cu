@@ -247,3 +247,79 @@ const char *fvattn_status_string(fvattn_status s)
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Routing without a caller-provided workspace.
+//
+// Some callers cannot call cudaMalloc at the point where they route: a
+// runtime that hands a plug-in only its input and output tensors, code that
+// runs under a memory-pool reservation that must not grow, or a process that
+// fixes its device footprint at start-up. For them the routing scratch -- the
+// status word and the pooled block means of Q and K -- lives in one array
+// compiled into this library, sized kNoAllocScratchBytes. Every GPU that
+// loads the library holds that array until the process exits.
+#include <mutex>
+
+namespace fvattn {
+
+constexpr size_t kNoAllocScratchBytes = 16u << 20;  // 16 MiB per device
+static __device__ __align__(256) uint8_t g_route_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void *g_scratch_addr[kMaxDevices];  // device address of g_route_scratch, per device, after set-up
+
+// The array's name in host code is only a stand-in for the device symbol;
+// kernels must get the device address, which is looked up once per device
+// (with that device current) and cached.
+cudaError_t route_scratch_address(void **out)
+{
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_route_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return cudaSuccess;
+}
+}  // namespace
+
+}  // namespace fvattn
+
+extern "C" fvattn_status fvattn_route_noalloc(const fvattn_problem *prob, const void *q, const void *k, float p,
+                                              int32_t k_min, int32_t *kv_cnt, int32_t *kv_idx, float *block_probs,
+                                              fvattn_stream_t stream)
+{
+    Geo g;
+    fvattn_status st = resolve(prob, &g);
+    if (st != FVATTN_OK) return st;
+    if (!(p > 0.f && p <= 1.f)) return FVATTN_ERR_INVALID_ARG;
+    if (k_min < 1 || k_min > g.nb) return FVATTN_ERR_INVALID_ARG;
+    if (!q || !k || !aligned16(q) || !aligned16(k)) return FVATTN_ERR_INVALID_ARG;
+    if (!kv_cnt || !kv_idx || !aligned4(kv_cnt) || !aligned4(kv_idx)) return FVATTN_ERR_INVALID_ARG;
+    if (block_probs && !aligned4(block_probs)) return FVATTN_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(g);
+    const size_t needed = L.kbarT + (size_t)g.BH * g.D * g.nbp * sizeof(float);
+    if (needed > kNoAllocScratchBytes) return FVATTN_ERR_WORKSPACE;
+    if (g.BH == 0) return FVATTN_OK;
+    void *scratch = nullptr;
+    if (route_scratch_address(&scratch) != cudaSuccess) return FVATTN_ERR_CUDA;
+    uint8_t *w = static_cast<uint8_t *>(scratch);
+    // Pooled means are written in full before they are read, so nothing needs
+    // clearing; the status word only collects flags nobody reads back here.
+    cudaStream_t s = (cudaStream_t)stream;
+    if (launch_pool(g, q, k, reinterpret_cast<float *>(w + L.qbar), reinterpret_cast<float *>(w + L.kbarT), s) !=
+        cudaSuccess)
+        return FVATTN_ERR_CUDA;
+    if (launch_score_select(g, reinterpret_cast<float *>(w + L.qbar), reinterpret_cast<float *>(w + L.kbarT), p,
+                            k_min, kv_cnt, kv_idx, block_probs, reinterpret_cast<uint32_t *>(w), s) != cudaSuccess)
+        return FVATTN_ERR_CUDA;
+    return FVATTN_OK;
+}

@@ -46,6 +46,7 @@ def _load():
         "fvattn_workspace_size": (sz, [P, i32]),
         "fvattn_workspace_init": (i32, [vp, sz, vp]),
         "fvattn_route": (i32, [P, vp, vp, f32, i32, vp, vp, vp, vp, sz, vp]),
+        "fvattn_route_noalloc": (i32, [P, vp, vp, f32, i32, vp, vp, vp, vp]),
         "fvattn_schedule": (i32, [P, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp]),
         "fvattn_sparse_attn": (i32, [P, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]),
         "fvattn_read_device_status": (i32, [vp, vp, ctypes.POINTER(ctypes.c_uint32)]),
@@ -60,7 +61,7 @@ def _load():
 
 _lib = _load()
 EXPORTED = ("fvattn_num_blocks", "fvattn_default_num_ctas", "fvattn_workspace_size", "fvattn_workspace_init",
-            "fvattn_route", "fvattn_schedule", "fvattn_sparse_attn", "fvattn_read_device_status",
+            "fvattn_route", "fvattn_route_noalloc", "fvattn_schedule", "fvattn_sparse_attn", "fvattn_read_device_status",
             "fvattn_status_string")
 
 
@@ -141,6 +142,21 @@ def route(geo: Geometry, q: torch.Tensor, k: torch.Tensor, p: float, k_min: int,
                            _ptr(kv_idx, torch.int32, "kv_idx"), _ptr(block_probs, torch.float32, "block_probs"),
                            _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
     _check(st, "fvattn_route")
+
+
+def route_noalloc(geo: Geometry, q: torch.Tensor, k: torch.Tensor, p: float, k_min: int,
+                  kv_cnt: torch.Tensor, kv_idx: torch.Tensor, block_probs: Optional[torch.Tensor] = None,
+                  stream=None):
+    """fvattn_route without a workspace, for callers that cannot allocate device
+    memory: the library's own fixed 16 MiB per-device array holds the scratch.
+    Calls that may overlap on the GPU race on that array; order them on one
+    stream, and make the first call on a device before any stream capture."""
+    prob = geo.problem()
+    st = _lib.fvattn_route_noalloc(ctypes.byref(prob), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+                                   float(p), int(k_min), _ptr(kv_cnt, torch.int32, "kv_cnt"),
+                                   _ptr(kv_idx, torch.int32, "kv_idx"),
+                                   _ptr(block_probs, torch.float32, "block_probs"), _stream(stream))
+    _check(st, "fvattn_route_noalloc")
 
 
 def schedule(geo: Geometry, kv_cnt: Optional[torch.Tensor], kv_idx: Optional[torch.Tensor], dense: bool,

@@ -184,6 +184,35 @@ FVATTN_API fvattn_status fvattn_sparse_attn(const fvattn_problem *prob, const vo
                                  int32_t dense, void *out, int64_t *cta_ns,
                                  void *ws, size_t ws_bytes, fvattn_stream_t stream);
 
+/*
+ * fvattn_route_noalloc -- fvattn_route for callers that cannot allocate device
+ * memory. The paper has no counterpart; it is a deployment convenience.
+ *
+ * Some callers cannot call cudaMalloc where they route: a runtime that hands
+ * a plug-in only its input and output tensors, code running under a memory
+ * pool reservation that must not grow, or a process whose device footprint
+ * is fixed at start-up. This entry point computes exactly what fvattn_route
+ * computes, with the same arguments except the workspace: its scratch (the
+ * pooled block means of Q and K) lives in a fixed 16 MiB array inside this
+ * library, which every GPU that loads the library holds until the process
+ * exits. The call allocates nothing (no cudaMalloc/cudaFree, no allocating
+ * library routine).
+ *   Limit: 4*(B*H*nb*D + B*H*D*round_up(nb,4)) plus 256 bytes must fit in
+ *   16 MiB (e.g. 24 heads x 120 blocks at D=128, or 40 x 360); larger problems
+ *   return FVATTN_ERR_WORKSPACE before anything is enqueued.
+ *   Set-up: the first call on each device looks up the array's device address
+ *   (with that device current) and caches it; make that first call before any
+ *   stream capture.
+ *   Sharing: every call on a device uses the same array, so calls that can
+ *   overlap on the GPU (different streams, no ordering between them) race and
+ *   may produce wrong lists; order them on one stream. Non-finite score rows
+ *   are repaired as in fvattn_route (kv_cnt == nb, NaN block_probs) but no
+ *   flag is reported.
+ */
+FVATTN_API fvattn_status fvattn_route_noalloc(const fvattn_problem *prob, const void *q, const void *k,
+                                              float p, int32_t k_min, int32_t *kv_cnt, int32_t *kv_idx,
+                                              float *block_probs, fvattn_stream_t stream);
+
 /* Synchronise `stream`, return the device status word's flags (FVATTN_FLAG_*)
  * in *flags, and clear them. Returns CUDA on a failed copy. */
 FVATTN_API fvattn_status fvattn_read_device_status(void *ws, fvattn_stream_t stream, uint32_t *flags);
