@@ -49,6 +49,8 @@ static fvattn_status resolve(const fvattn_problem *p, Geo *g)
     const long long bp = (long long)p->blk_t * p->blk_h * p->blk_w;
     if (!(bp == 256 && p->blk_t % 2 == 0) && bp != 64) return FVATTN_ERR_UNSUPPORTED;
     if (p->blk_w > 256 || p->blk_h > 256 || p->blk_t > 256) return FVATTN_ERR_UNSUPPORTED;
+    // the attention kernel keeps one column mask per extent along each block axis
+    if (p->blk_w + p->blk_h + (bp == 256 ? p->blk_t / 2 : p->blk_t) > 40) return FVATTN_ERR_UNSUPPORTED;
     Geo G;
     G.B = p->B;
     G.H = p->H;

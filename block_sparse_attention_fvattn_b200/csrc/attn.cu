@@ -21,35 +21,53 @@
 //
 // Roles (384 threads = 3 warpgroups, one CTA per SM):
 //   warp 0      TMA producer: Q halves, K and V sub-tiles into rings
-//   warp 1      MMA issuer: S_h = Q_h K^T (A, B from shared memory) and
-//               O_h += P_h V (A = P from tensor memory, B = V from shared
-//               memory, MN-major); owns the TMEM allocation
+//   warp 1      MMA issuer (one thread) and owner of the TMEM allocation:
+//               S = Q_h K^T (A and B from shared memory) and
+//               O_h += P_h V (A = P_h from TMEM, B = V from shared memory, MN-major)
 //   warps 2-3   idle (they only return registers)
 //   warps 4-7   softmax + epilogue for query half 0
 //   warps 8-11  softmax + epilogue for query half 1
 // A warp reaches TMEM lanes 32*(warp % 4) .. +31, so each softmax warpgroup
 // covers the 128 rows of its half (row = 32*(warp%4) + lane) and holds a
 // whole 128-column score row in registers.
-// TMEM columns: S_0 [0,128) S_1 [128,256) O_0 [256,256+D) O_1 [256+D, 256+2D);
-// P_h (bf16 pairs) overwrites the first BKV/2 columns of S_h. The online
-// softmax rescales O lazily, only when a row maximum grows by more than 2^8.
+//
+// TMEM (512 columns x 128 lanes): one S buffer [0,128) shared by both halves,
+// P_0 [128,192) and P_1 [192,256) (bf16 pairs), O_0 [256,256+D), O_1 after it.
+// S is free again as soon as the softmax warpgroup has copied it into
+// registers, so the next QK never waits for a PV to finish; the MMA order per
+// sub-tile k is PV_0(k), QK_0(k+1), PV_1(k), QK_1(k+1), which lets one half's
+// softmax overlap the other half's products. The online softmax rescales O
+// lazily, only when a row maximum grows by more than 2^8.
 #include "common.cuh"
+#include "exp2_poly.h"
 #include "internal.h"
+
+// Pairs of softmax columns (out of every 16) whose exponential is evaluated
+// with the polynomial on the FMA/ALU pipes instead of the MUFU unit. Off by
+// default: measured on B200 the MUFU unit is not the limit of this kernel, and
+// the extra FMA/ALU instructions slow the MMA issue warp that shares their
+// sub-partitions (Wan-5B-like layer: 724 / 687 / 650 TFLOPS for 0 / 4 / 8).
+#ifndef FV_POLY_PAIRS
+#define FV_POLY_PAIRS 0
+#endif
 
 namespace fvattn {
 
 constexpr int kNK = 2;  // K ring stages
-constexpr int kNV = 2;  // V ring stages
+constexpr int kNV = 3;  // V ring stages
 constexpr int kThreads = 384;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Register split between warpgroups (setmaxnreg). The kernel is launched with
 // kLaunchRegs per thread (checked on the host before every launch); the
 // producer/MMA warpgroup gives registers back and the two softmax
-// warpgroups take them: 128*kRegsLow + 256*kRegsHigh == 384*kLaunchRegs.
+// warpgroups take them: 128*low + 256*high <= 384*kLaunchRegs.
 constexpr int kLaunchRegs = 168;
-constexpr int kRegsLow = 56;
-constexpr int kRegsHigh = 224;
-static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kLaunchRegs, "register split exceeds the launch budget");
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+template <int D, int BKV>
+struct RegSplit {
+    static constexpr int kLow = 72;
+    static constexpr int kHigh = BKV == 64 ? 208 : 216;
+    static_assert(128 * kLow + 256 * kHigh <= kThreads * kLaunchRegs, "register split exceeds the launch budget");
+};
 
 template <int D, int BKV>
 struct AttnLayout {
@@ -61,14 +79,22 @@ struct AttnLayout {
     static constexpr int kV = kK + kNK * kDH * kKVSlab;
     static constexpr int kMask = kV + kNV * kDH * kKVSlab;
     static constexpr int kMaskWords = BKV / 32;
-    static constexpr int kBar = kMask + BKV * kMaskWords * 4;
+    // per-axis column masks: entry v-1 of each axis keeps the columns whose
+    // coordinate along that axis is < v; blk_w + blk_h + sub_t <= kMaskEntries
+    static constexpr int kMaskEntries = 40;
+    static constexpr int kBar = kMask + kMaskEntries * kMaskWords * 4;
     // barrier indices
     static constexpr int bQFull = 0, bQEmpty = 2, bKFull = 4, bKEmpty = bKFull + kNK, bVFull = bKEmpty + kNK,
-                         bVEmpty = bVFull + kNV, bSFull = bVEmpty + kNV, bPFull = bSFull + 2, bOFull = bPFull + 2,
-                         bOEmpty = bOFull + 2, bPVDone = bOEmpty + 2, bDrain = bPVDone + 2, kNumBars = bDrain + 1;
+                         bVEmpty = bVFull + kNV, bSFull = bVEmpty + kNV, bSFree = bSFull + 2, bPFull = bSFree + 1,
+                         bPFree = bPFull + 2, bOFull = bPFree + 2, bOEmpty = bOFull + 2, bDrain = bOEmpty + 2,
+                         kNumBars = bDrain + 1;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 64;
     static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
+    // TMEM columns
+    static constexpr uint32_t kTmS = 0, kTmP = 128, kTmO = 256;
+    static uint32_t __device__ __forceinline__ tm_p(int h) { return kTmP + 64u * (uint32_t)h; }
+    static uint32_t __device__ __forceinline__ tm_o(int h) { return kTmO + (uint32_t)(D * h); }
 };
 
 struct Unit {
@@ -147,6 +173,31 @@ struct UnitSeq {
     }
 };
 
+// Two exponentials 2^a (a = packed pair) on the FMA/ALU pipes:
+// a = j + f with j = round(a) (1.5*2^23 rounding constant), f in [-1/2, 1/2],
+// 2^a = 2^j * p(f) with p the degree-3 minimax polynomial of exp2_poly.h; 2^j is
+// applied by adding j to the exponent field. Arguments below -126 give values
+// below 2^-126 (a denormal or zero pattern), never NaN.
+__device__ __forceinline__ void exp2_poly_x2(uint64_t a, float &p0, float &p1)
+{
+    float a0, a1;
+    f2_unpack(a, a0, a1);
+    // p(f) lies in [0.70, 1.42], i.e. its biased exponent is 126 or 127, so adding
+    // j >= -126 to the exponent field can neither wrap nor reach the sign bit
+    a0 = fmaxf(a0, -126.0f);
+    a1 = fmaxf(a1, -126.0f);
+    const float t0 = a0 + 12582912.0f, t1 = a1 + 12582912.0f;  // round to nearest integer
+    const float f0 = a0 - (t0 - 12582912.0f), f1 = a1 - (t1 - 12582912.0f);
+    const uint64_t f = f2_pack(f0, f1);
+    uint64_t q = f2_fma(f2_pack(FV_EXP2_C3, FV_EXP2_C3), f, f2_pack(FV_EXP2_C2, FV_EXP2_C2));
+    q = f2_fma(q, f, f2_pack(FV_EXP2_C1, FV_EXP2_C1));
+    q = f2_fma(q, f, f2_pack(FV_EXP2_C0, FV_EXP2_C0));
+    float q0, q1;
+    f2_unpack(q, q0, q1);
+    p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+    p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
 template <int D, int BKV>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -160,7 +211,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw = smem_u32(attn_smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
     uint8_t *gbase = attn_smem_raw + (sbase - raw);
-    const uint32_t *mask_tab = reinterpret_cast<const uint32_t *>(gbase + L::kMask);
+    const uint32_t *mask_w = reinterpret_cast<const uint32_t *>(gbase + L::kMask);
+    const uint32_t *mask_h = mask_w + g.bw * L::kMaskWords;
+    const uint32_t *mask_t = mask_h + g.bh * L::kMaskWords;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + L::kMisc);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + L::kMisc + 16);
     auto bar = [&](int idx) -> uint32_t { return sbase + L::kBar + 8u * (uint32_t)idx; };
@@ -168,19 +221,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t t_start = globaltimer_ns();
 
-    // ---- set-up: column-validity table, barriers, TMEM
+    // ---- set-up: per-axis column masks, barriers, TMEM
     {
         uint32_t *tab = reinterpret_cast<uint32_t *>(gbase + L::kMask);
-        for (int pat = threadIdx.x; pat < BKV; pat += blockDim.x) {
-            const int wv = pat % g.bw + 1, hv = (pat / g.bw) % g.bh + 1, tv = pat / (g.bw * g.bh) + 1;
+        const int n_ent = g.bw + g.bh + g.subt;
+        for (int ent = threadIdx.x; ent < n_ent; ent += blockDim.x) {
+            const int axis = ent < g.bw ? 0 : (ent < g.bw + g.bh ? 1 : 2);
+            const int v = 1 + (axis == 0 ? ent : (axis == 1 ? ent - g.bw : ent - g.bw - g.bh));
             for (int w = 0; w < L::kMaskWords; ++w) {
                 uint32_t word = 0;
                 for (int b = 0; b < 32; ++b) {
                     const int c = w * 32 + b;
-                    const int tt = c / (g.bh * g.bw), yy = (c / g.bw) % g.bh, xx = c % g.bw;
-                    if (xx < wv && yy < hv && tt < tv) word |= 1u << b;
+                    const int coord = axis == 0 ? c % g.bw : (axis == 1 ? (c / g.bw) % g.bh : c / (g.bh * g.bw));
+                    if (coord < v) word |= 1u << b;
                 }
-                tab[pat * L::kMaskWords + w] = word;
+                tab[ent * L::kMaskWords + w] = word;
             }
         }
     }
@@ -188,7 +243,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         for (int b = 0; b < L::kNumBars; ++b) {
             uint32_t cnt = 1;
-            if (b == L::bPFull || b == L::bPFull + 1 || b == L::bOEmpty || b == L::bOEmpty + 1) cnt = 128;
+            if (b == L::bSFree || b == L::bPFull || b == L::bPFull + 1 || b == L::bOEmpty || b == L::bOEmpty + 1)
+                cnt = 128;  // arrived on by all 128 threads of a softmax warpgroup
             mbar_init(bar(b), cnt);
         }
         fence_mbar_init();
@@ -217,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t kTileBytes = (uint32_t)L::kDH * BKV * 128u;
     const uint32_t q_bytes = (uint32_t)L::kDH * (uint32_t)g.rows * 128u;
 
-    if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+    if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(RegSplit<D, BKV>::kLow));
     if (warp == 0) {
         // ================= TMA producer =================
         if (lane == 0) {
@@ -291,66 +347,71 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(128, BKV, false);
             constexpr uint32_t idesc_pv = idesc_bf16(128, D, true);
-            int kc = 0, vc = 0;
-            // one parity bit per query half for each barrier pair, and one
-            // "committed but not yet waited for" bit per half
-            uint32_t ph_q = 0, ph_p = 0, ph_pv = 0, ph_oe = 0, pv_pend = 0, o_pend = 0;
+            // descriptors of the first slab of each region; every other operand
+            // is a fixed byte offset from it (added to the start-address field)
+            const uint64_t q_desc = sdesc_sw128(sbase + L::kQ, 16, 1024);
+            const uint64_t k_desc = sdesc_sw128(sbase + L::kK, 16, 1024);
+            const uint64_t v_desc = sdesc_sw128(sbase + L::kV, L::kKVSlab, 1024);
+            int kc = 0, vc = 0, qk_count = 0;
+            uint32_t ph_q = 0, ph_p = 0, ph_oe = 0, o_pend = 0;
             bool ok = true;
-            // S_h = Q_h K^T over D in K=16 steps; Q and K slabs are K-major, 128B swizzle
+            // S = Q_h K^T over D in K=16 steps; Q and K slabs are K-major, 128B swizzle
             auto issue_qk = [&](int h, int ks) {
-                const uint32_t d_tmem = tmem + (uint32_t)(h * 128);
+                const uint64_t qa = q_desc + (uint64_t)((h * L::kDH * L::kQSlab) >> 4);
+                const uint64_t kb = k_desc + (uint64_t)((ks * L::kDH * L::kKVSlab) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const int dh = kk >> 2, within = kk & 3;
-                    const uint32_t a = sbase + L::kQ + (h * L::kDH + dh) * L::kQSlab + within * 32;
-                    const uint32_t b = sbase + L::kK + (ks * L::kDH + dh) * L::kKVSlab + within * 32;
-                    umma_ss(d_tmem, sdesc_sw128(a, 16, 1024), sdesc_sw128(b, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+                    const uint32_t off_a = ((kk >> 2) * L::kQSlab + (kk & 3) * 32) >> 4;
+                    const uint32_t off_b = ((kk >> 2) * L::kKVSlab + (kk & 3) * 32) >> 4;
+                    umma_ss(tmem + L::kTmS, qa + off_a, kb + off_b, idesc_qk, kk > 0 ? 1u : 0u);
                 }
             };
-            // O_h (+)= P_h V over the sub-tile in K=16 steps; P from TMEM, V MN-major
+            // O_h (+)= P_h V over the sub-tile in K=16 steps; P_h from TMEM, V MN-major
             auto issue_pv = [&](int h, int vs, bool accumulate) {
-                const uint32_t d_tmem = tmem + 256u + (uint32_t)(h * D);
+                const uint64_t vb = v_desc + (uint64_t)((vs * L::kDH * L::kKVSlab) >> 4);
+                const uint32_t d_tmem = tmem + L::tm_o(h), a_tmem = tmem + L::tm_p(h);
 #pragma unroll
-                for (int kk = 0; kk < BKV / 16; ++kk) {
-                    const uint32_t a_tmem = tmem + (uint32_t)(h * 128 + kk * 8);
-                    const uint32_t b = sbase + L::kV + (vs * L::kDH) * L::kKVSlab + kk * 16 * 128;
-                    umma_ts(d_tmem, a_tmem, sdesc_sw128(b, L::kKVSlab, 1024), idesc_pv,
+                for (int kk = 0; kk < BKV / 16; ++kk)
+                    umma_ts(d_tmem, a_tmem + kk * 8, vb + (uint64_t)((kk * 16 * 128) >> 4), idesc_pv,
                             (accumulate || kk > 0) ? 1u : 0u);
-                }
             };
             auto wait_half = [&](int base, uint32_t &ph, int h) -> bool {
                 const bool r = mbar_wait(bar(base + h), (ph >> h) & 1u, abort_flag);
                 ph ^= 1u << h;
                 return r;
             };
+            // S is shared: a QK may only overwrite it once the previous S has been
+            // copied out by its softmax warpgroup
+            auto qk = [&](int h, int ks) -> bool {
+                if (qk_count > 0 && !mbar_wait(bar(L::bSFree), (qk_count - 1) & 1, abort_flag)) return false;
+                tc_fence_after();
+                issue_qk(h, ks);
+                umma_commit(bar(L::bSFull + h));
+                ++qk_count;
+                return true;
+            };
             int u;
             for (long long idx = 0; ok && seq.get(idx, u); ++idx) {
                 const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
                 for (int h = 0; h < U.nh && ok; ++h) ok = wait_half(L::bQFull, ph_q, h);
                 if (!ok) break;
-                // first S tiles
                 int ks = kc % kNK;
                 if (!mbar_wait(bar(L::bKFull + ks), (kc / kNK) & 1, abort_flag)) break;
-                tc_fence_after();
                 for (int h = 0; h < U.nh && ok; ++h) {
-                    if ((pv_pend >> h) & 1u) {  // S_h is free once the last PV that read P_h is done
-                        ok = wait_half(L::bPVDone, ph_pv, h);
-                        pv_pend &= ~(1u << h);
-                        tc_fence_after();
-                    }
-                    if (!ok) break;
-                    issue_qk(h, ks);
-                    umma_commit(bar(L::bSFull + h));
+                    ok = qk(h, ks);
+                    if (ok && U.nkv == 1) umma_commit(bar(L::bQEmpty + h));
                 }
                 if (!ok) break;
                 umma_commit(bar(L::bKEmpty + ks));
                 ++kc;
-                if (U.nkv == 1)
-                    for (int h = 0; h < U.nh; ++h) umma_commit(bar(L::bQEmpty + h));
+                // per sub-tile k: PV_0(k), QK_0(k+1), PV_1(k), QK_1(k+1)
                 for (int k = 0; k < U.nkv && ok; ++k) {
+                    const bool next = k + 1 < U.nkv;
                     const int vs = vc % kNV;
                     if (!mbar_wait(bar(L::bVFull + vs), (vc / kNV) & 1, abort_flag)) { ok = false; break; }
+                    ks = kc % kNK;
                     for (int h = 0; h < U.nh && ok; ++h) {
+                        const bool last_h = h == U.nh - 1;
                         ok = wait_half(L::bPFull, ph_p, h);
                         if (ok && k == 0 && ((o_pend >> h) & 1u)) {  // previous unit's epilogue read O_h
                             ok = wait_half(L::bOEmpty, ph_oe, h);
@@ -359,34 +420,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!ok) break;
                         tc_fence_after();
                         issue_pv(h, vs, k > 0);
-                        umma_commit(bar(L::bPVDone + h));
-                        pv_pend |= 1u << h;
-                        if (k == U.nkv - 1) {
+                        umma_commit(bar(L::bPFree + h));
+                        if (!next) {
                             umma_commit(bar(L::bOFull + h));
                             o_pend |= 1u << h;
                         }
+                        if (last_h) umma_commit(bar(L::bVEmpty + vs));
+                        if (next) {
+                            if (h == 0 && !mbar_wait(bar(L::bKFull + ks), (kc / kNK) & 1, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            ok = qk(h, ks);
+                            if (!ok) break;
+                            if (k + 2 == U.nkv) umma_commit(bar(L::bQEmpty + h));
+                            if (last_h) umma_commit(bar(L::bKEmpty + ks));
+                        }
                     }
                     if (!ok) break;
-                    umma_commit(bar(L::bVEmpty + vs));
                     ++vc;
-                    if (k + 1 < U.nkv) {
-                        ks = kc % kNK;
-                        if (!mbar_wait(bar(L::bKFull + ks), (kc / kNK) & 1, abort_flag)) { ok = false; break; }
-                        tc_fence_after();
-                        for (int h = 0; h < U.nh && ok; ++h) {
-                            ok = wait_half(L::bPVDone, ph_pv, h);
-                            pv_pend &= ~(1u << h);
-                            if (!ok) break;
-                            tc_fence_after();
-                            issue_qk(h, ks);
-                            umma_commit(bar(L::bSFull + h));
-                        }
-                        if (!ok) break;
-                        umma_commit(bar(L::bKEmpty + ks));
-                        ++kc;
-                        if (k + 2 == U.nkv)
-                            for (int h = 0; h < U.nh; ++h) umma_commit(bar(L::bQEmpty + h));
-                    }
+                    if (next) ++kc;
                 }
             }
             // every MMA issued must finish before TMEM is released
@@ -395,17 +448,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= 4) {
         // ================= softmax + epilogue =================
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(RegSplit<D, BKV>::kHigh));
         const int h = (warp - 4) >> 2;
         const int wq = warp & 3;
         const int row = wq * 32 + lane;
         const uint32_t t_lane = (uint32_t)(wq * 32) << 16;
-        const uint32_t tS = tmem + t_lane + (uint32_t)(h * 128);
-        const uint32_t tO = tmem + t_lane + 256u + (uint32_t)(h * D);
+        const uint32_t tS = tmem + t_lane + L::kTmS;
+        const uint32_t tP = tmem + t_lane + L::tm_p(h);
+        const uint32_t tO = tmem + t_lane + L::tm_o(h);
         const float sl2 = g.scale * 1.4426950408889634f;
         // this thread's query row inside a sub-tile
         const int r_t = row / (g.bh * g.bw), r_y = (row / g.bw) % g.bh, r_x = row % g.bw;
-        int sf = 0, of = 0;
+        int sf = 0, of = 0, pw = 0;  // S tiles received, O tiles received, P tiles written
         bool ok = true;
         int u;
         for (long long idx = 0; ok && seq.get(idx, u); ++idx) {
@@ -414,38 +468,52 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int qt = U.it * g.bt + h * g.subt + r_t, qy = U.iy * g.bh + r_y, qx = U.ix * g.bw + r_x;
             const bool row_valid = row < g.rows && qt < g.T && qy < g.Hg && qx < g.W;
             float m = -INFINITY, l = 0.f;
-            TileCursor cur;
+            int e = 0, s_sub = 0;
+            int j = U.list ? __ldg(U.list) : 0;
             for (int k = 0; k < U.nkv; ++k) {
-                const int j = cur.block(U);
+                // the list entry after this one is loaded now and used next iteration
+                const int j_next = (U.list && e + 1 < U.cnt) ? __ldg(U.list + e + 1) : e + 1;
                 const int jt = j / (g.nbh * g.nbw), jy = (j / g.nbw) % g.nbh, jx = j % g.nbw;
                 const int wv = min(g.bw, g.W - jx * g.bw), hv = min(g.bh, g.Hg - jy * g.bh);
-                const int tv = min(g.subt, g.T - (jt * g.bt + cur.s * g.subt));
+                const int tv = min(g.subt, g.T - (jt * g.bt + s_sub * g.subt));
                 const bool full = (wv == g.bw) && (hv == g.bh) && (tv == g.subt);
                 if (!mbar_wait(bar(L::bSFull + h), sf & 1, abort_flag)) { ok = false; break; }
                 ++sf;
                 tc_fence_after();
+                // all BKV columns in one batch, one wait; the register fences keep
+                // every use of the loaded values after the wait
+                uint32_t r[BKV];
+#pragma unroll
+                for (int c = 0; c < BKV / 32; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(r + c * 32));
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < BKV / 32; ++c) reg_fence32(r + c * 32);
+                // S is in registers: the next QK may overwrite it
+                tc_fence_before();
+                mbar_arrive(bar(L::bSFree));
                 float x[BKV];
 #pragma unroll
-                for (int c = 0; c < BKV / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tS + c * 32, r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int v = 0; v < 32; ++v) x[c * 32 + v] = __uint_as_float(r[v]);
-                }
+                for (int c = 0; c < BKV; ++c) x[c] = __uint_as_float(r[c]);
                 if (!full) {
-                    const uint32_t *mw = mask_tab + (((tv - 1) * g.bh + (hv - 1)) * g.bw + (wv - 1)) * L::kMaskWords;
 #pragma unroll
                     for (int w = 0; w < L::kMaskWords; ++w) {
-                        const uint32_t word = mw[w];
+                        const uint32_t word = mask_w[(wv - 1) * L::kMaskWords + w] &
+                                              mask_h[(hv - 1) * L::kMaskWords + w] &
+                                              mask_t[(tv - 1) * L::kMaskWords + w];
 #pragma unroll
                         for (int b = 0; b < 32; ++b)
                             if (!((word >> b) & 1u)) x[w * 32 + b] = -INFINITY;
                     }
                 }
-                float mx = x[0];
+                // row maximum: 8 independent chains of three-input max, then a tree
+                float m8[8];
 #pragma unroll
-                for (int c = 1; c < BKV; ++c) mx = fmaxf(mx, x[c]);
+                for (int q8 = 0; q8 < 8; ++q8) m8[q8] = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < BKV; c += 16)
+#pragma unroll
+                    for (int q8 = 0; q8 < 8; ++q8) m8[q8] = max3f(m8[q8], x[c + 2 * q8], x[c + 2 * q8 + 1]);
+                const float mx = fmaxf(max3f(m8[0], m8[1], m8[2]), max3f(max3f(m8[3], m8[4], m8[5]), m8[6], m8[7]));
                 const float mt = mx * sl2;
                 float alpha = 1.0f;
                 bool rescale = false;
@@ -460,22 +528,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                         l *= alpha;
                     }
                 }
-                float sum = 0.f;
+                // P_h and O_h are free once the PV of this half's previous sub-tile is done
+                if (pw > 0 && !mbar_wait(bar(L::bPFree + h), (pw - 1) & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                // p = 2^(x*scale*log2e - m); packed fp32x2 FMA/ADD, MUFU ex2 or the
+                // polynomial, bf16 pairs into P_h
+                const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m, -m);
+                uint64_t s4[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
                 for (int c = 0; c < BKV / 32; ++c) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int q2 = 0; q2 < 16; ++q2) {
-                        const float p0 = ex2_approx(fmaf(x[c * 32 + 2 * q2], sl2, -m));
-                        const float p1 = ex2_approx(fmaf(x[c * 32 + 2 * q2 + 1], sl2, -m));
-                        sum += p0 + p1;
+                        const uint64_t a = f2_fma(f2_pack(x[c * 32 + 2 * q2], x[c * 32 + 2 * q2 + 1]), sl2x2, negm2);
+                        float p0, p1;
+                        if ((q2 & 7) < FV_POLY_PAIRS / 2) {
+                            exp2_poly_x2(a, p0, p1);
+                        } else {
+                            float a0, a1;
+                            f2_unpack(a, a0, a1);
+                            p0 = ex2_approx(a0);
+                            p1 = ex2_approx(a1);
+                        }
+                        s4[q2 & 3] = f2_add(s4[q2 & 3], f2_pack(p0, p1));
                         pk[q2] = pack_bf16x2(p0, p1);
                     }
-                    tmem_st16(tS + c * 16, pk);
+                    tmem_st16(tP + c * 16, pk);
+                }
+                float sum;
+                {
+                    const uint64_t t = f2_add(f2_add(s4[0], s4[1]), f2_add(s4[2], s4[3]));
+                    float t0, t1;
+                    f2_unpack(t, t0, t1);
+                    sum = t0 + t1;
                 }
                 if (rescale) {
-                    // O_h holds the sum up to the previous sub-tile (its PV finished
-                    // before this S was produced); bring it to the new row maximum.
+                    // O_h holds the sum up to the previous sub-tile (its PV is done);
+                    // bring it to the new row maximum
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t o[32];
@@ -489,8 +578,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(bar(L::bPFull + h));
+                ++pw;
                 l += sum;
-                cur.advance(g, U);
+                if (g.nsub == 2 && s_sub == 0 && jt * g.bt + g.subt < g.T) {
+                    s_sub = 1;
+                } else {
+                    s_sub = 0;
+                    ++e;
+                    j = j_next;
+                }
             }
             if (!ok) break;
             // epilogue: O / l -> bf16, raster order, valid rows only
@@ -582,7 +678,8 @@ static cudaError_t launch_attn_t(const Geo &g, const CUtensorMap &mq, const CUte
     if (err != cudaSuccess) return err;
     // the setmaxnreg split must fit in what the launch provides, or the
     // softmax warpgroups would wait for registers forever
-    if (fa.numRegs * kThreads < 128 * kRegsLow + 256 * kRegsHigh) return cudaErrorInvalidConfiguration;
+    if (fa.numRegs * kThreads < 128 * RegSplit<D, BKV>::kLow + 256 * RegSplit<D, BKV>::kHigh)
+        return cudaErrorInvalidConfiguration;
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (err != cudaSuccess) return err;
     kern<<<grid, kThreads, L::kAlloc, stream>>>(mq, mk, mv, g, kv_cnt, kv_idx, work, cta_range, dense,

@@ -10,10 +10,11 @@
 //   s = scale * Qbar_i . Kbar_j, softmax, Top-p with a Top-k floor, diagonal
 //   repair and ascending compaction (ai-feeds.com FVAttn summary, "Key
 //   modules" 1; hotpaper.ai abstract). The nb x nb score matrix never leaves
-//   shared memory. Selection is exact in fp32: an order-preserving integer key
-//   of each score and a bisection over the key space find the score at the
-//   Top-p boundary (by probability mass) and, if the floor binds, at rank m;
-//   ties at the boundary go to the lower block index.
+//   shared memory. One warp owns one row. Selection is exact in fp32: an
+//   order-preserving integer key of each score and a 4-ary search over the key
+//   space find the score at the Top-p boundary (by probability mass) and, if
+//   the floor binds, at rank m; ties at the boundary go to the lower block
+//   index.
 #include "common.cuh"
 #include "internal.h"
 
@@ -104,15 +105,9 @@ __global__ void __launch_bounds__(256) pool_kernel(Geo g, const __nv_bfloat16 *_
 
 // ---------------------------------------------------------------------------
 // K2
-constexpr int kSelRows = 16;  // query blocks per CTA (rows of the score tile)
+constexpr int kSelRows = 8;  // query blocks per CTA (rows of the score tile), one per warp
 
 __device__ __forceinline__ float warp_sum(float v)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-    return v;
-}
-__device__ __forceinline__ int warp_sum_i(int v)
 {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
@@ -165,7 +160,7 @@ __global__ void __launch_bounds__(256) score_select_kernel(Geo g, const float *_
     }
     __syncthreads();
 
-    // ---- block scores: each thread owns 4 consecutive key blocks x 16 rows
+    // ---- block scores: each thread owns 4 consecutive key blocks x kSelRows rows
     const float *kb = kbarT + (size_t)bh * D * nbp;
     for (int c0 = threadIdx.x * 4; c0 < nbp; c0 += blockDim.x * 4) {
         float acc[kSelRows][4];
@@ -173,7 +168,7 @@ __global__ void __launch_bounds__(256) score_select_kernel(Geo g, const float *_
         for (int r = 0; r < kSelRows; ++r)
 #pragma unroll
             for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
-#pragma unroll 4
+#pragma unroll 8
         for (int d = 0; d < D; ++d) {
             const float4 kv = __ldg(reinterpret_cast<const float4 *>(kb + (size_t)d * nbp + c0));
             const float4 *qv = reinterpret_cast<const float4 *>(qsT + d * kSelRows);
@@ -269,16 +264,34 @@ __global__ void __launch_bounds__(256) score_select_kernel(Geo g, const float *_
             all_sel = true;
         } else {
             const float target = p * z;
-            // largest key t with mass(key >= t) >= target
+            // largest key t with mass(key >= t) >= target: 4-ary search, three
+            // independent reductions per step
             uint32_t lo = kmin, hi = kmax + 1u;
             while (hi - lo > 1u) {
-                const uint32_t mid = lo + ((hi - lo) >> 1);
-                float mass = 0.f;
+                const uint32_t q4 = (hi - lo) >> 2;
+                const uint32_t t1 = lo + (q4 ? q4 : 1u), t2 = lo + (q4 ? 2u * q4 : 1u),
+                               t3 = lo + (q4 ? 3u * q4 : 1u);
+                float m1 = 0.f, m2 = 0.f, m3 = 0.f;
 #pragma unroll
-                for (int e = 0; e < EPL; ++e) mass += (key[e] >= mid) ? pv[e] : 0.f;
-                mass = warp_sum(mass);
-                if (mass >= target) lo = mid;
-                else hi = mid;
+                for (int e = 0; e < EPL; ++e) {
+                    m1 += (key[e] >= t1) ? pv[e] : 0.f;
+                    m2 += (key[e] >= t2) ? pv[e] : 0.f;
+                    m3 += (key[e] >= t3) ? pv[e] : 0.f;
+                }
+                m1 = warp_sum(m1);
+                m2 = warp_sum(m2);
+                m3 = warp_sum(m3);
+                if (m3 >= target) {
+                    lo = t3;
+                } else if (m2 >= target) {
+                    lo = t2;
+                    hi = t3;
+                } else if (m1 >= target) {
+                    lo = t1;
+                    hi = t2;
+                } else {
+                    hi = t1;
+                }
             }
             const uint32_t kp = lo;
             float mass_gt = 0.f, p_eq = 0.f;
@@ -291,8 +304,8 @@ __global__ void __launch_bounds__(256) score_select_kernel(Geo g, const float *_
                 if (key[e] == kp) p_eq = pv[e];
             }
             mass_gt = warp_sum(mass_gt);
-            cnt_gt = warp_sum_i(cnt_gt);
-            n_eq = warp_sum_i(n_eq);
+            cnt_gt = (int)__reduce_add_sync(0xFFFFFFFFu, (uint32_t)cnt_gt);
+            n_eq = (int)__reduce_add_sync(0xFFFFFFFFu, (uint32_t)n_eq);
             p_eq = warp_max(p_eq);
             // blocks tied at the boundary enter one at a time, lowest index first
             float accm = mass_gt;
@@ -309,22 +322,39 @@ __global__ void __launch_bounds__(256) score_select_kernel(Geo g, const float *_
                 kap = kp;
                 ntie = n;
             } else {
-                // Top-k floor binds: boundary key of rank m
+                // Top-k floor binds: boundary key of rank m (4-ary search on counts)
                 uint32_t lo2 = kmin, hi2 = kp + 1u;
                 while (hi2 - lo2 > 1u) {
-                    const uint32_t mid = lo2 + ((hi2 - lo2) >> 1);
-                    int c = 0;
+                    const uint32_t q4 = (hi2 - lo2) >> 2;
+                    const uint32_t t1 = lo2 + (q4 ? q4 : 1u), t2 = lo2 + (q4 ? 2u * q4 : 1u),
+                                   t3 = lo2 + (q4 ? 3u * q4 : 1u);
+                    uint32_t c1 = 0, c2 = 0, c3 = 0;
 #pragma unroll
-                    for (int e = 0; e < EPL; ++e) c += (key[e] >= mid) ? 1 : 0;
-                    c = warp_sum_i(c);
-                    if (c >= m) lo2 = mid;
-                    else hi2 = mid;
+                    for (int e = 0; e < EPL; ++e) {
+                        c1 += (key[e] >= t1) ? 1u : 0u;
+                        c2 += (key[e] >= t2) ? 1u : 0u;
+                        c3 += (key[e] >= t3) ? 1u : 0u;
+                    }
+                    c1 = __reduce_add_sync(0xFFFFFFFFu, c1);
+                    c2 = __reduce_add_sync(0xFFFFFFFFu, c2);
+                    c3 = __reduce_add_sync(0xFFFFFFFFu, c3);
+                    if (c3 >= (uint32_t)m) {
+                        lo2 = t3;
+                    } else if (c2 >= (uint32_t)m) {
+                        lo2 = t2;
+                        hi2 = t3;
+                    } else if (c1 >= (uint32_t)m) {
+                        lo2 = t1;
+                        hi2 = t2;
+                    } else {
+                        hi2 = t1;
+                    }
                 }
                 kap = lo2;
                 int c_gt = 0;
 #pragma unroll
                 for (int e = 0; e < EPL; ++e) c_gt += (key[e] > kap) ? 1 : 0;
-                c_gt = warp_sum_i(c_gt);
+                c_gt = (int)__reduce_add_sync(0xFFFFFFFFu, (uint32_t)c_gt);
                 ntie = m - c_gt;
             }
         }
