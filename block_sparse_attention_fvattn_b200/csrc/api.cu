@@ -82,6 +82,8 @@ static fvattn_status resolve(const fvattn_problem *p, Geo *g)
         G.rows = 64;
     }
     G.scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / sqrtf((float)G.D);
+    G.fd_nbw = make_fastdiv((uint32_t)G.nbw);
+    G.fd_hw = make_fastdiv((uint32_t)(G.nbh * G.nbw));
     *g = G;
     return FVATTN_OK;
 }

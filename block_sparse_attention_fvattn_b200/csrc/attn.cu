@@ -21,10 +21,12 @@
 //
 // Roles (384 threads = 3 warpgroups, one CTA per SM):
 //   warp 0      TMA producer: Q halves, K and V sub-tiles into rings
-//   warp 1      MMA issuer (one thread) and owner of the TMEM allocation:
-//               S = Q_h K^T (A and B from shared memory) and
-//               O_h += P_h V (A = P_h from TMEM, B = V from shared memory, MN-major)
-//   warps 2-3   idle (they only return registers)
+//   warp 1      QK issuer (one thread) and owner of the TMEM allocation:
+//               S = Q_h K^T (A and B from shared memory)
+//   warp 2      PV issuer (one thread): O_h += P_h V (A = P_h from TMEM,
+//               B = V from shared memory, MN-major). Two issuing threads keep
+//               the tensor core fed while either one waits on a barrier.
+//   warp 3      idle (it only returns registers)
 //   warps 4-7   softmax + epilogue for query half 0
 //   warps 8-11  softmax + epilogue for query half 1
 // A warp reaches TMEM lanes 32*(warp % 4) .. +31, so each softmax warpgroup
@@ -34,9 +36,8 @@
 // TMEM (512 columns x 128 lanes): one S buffer [0,128) shared by both halves,
 // P_0 [128,192) and P_1 [192,256) (bf16 pairs), O_0 [256,256+D), O_1 after it.
 // S is free again as soon as the softmax warpgroup has copied it into
-// registers, so the next QK never waits for a PV to finish; the MMA order per
-// sub-tile k is PV_0(k), QK_0(k+1), PV_1(k), QK_1(k+1), which lets one half's
-// softmax overlap the other half's products. The online softmax rescales O
+// registers, so the next QK never waits for a PV to finish, and one half's
+// softmax overlaps the other half's products. The online softmax rescales O
 // lazily, only when a row maximum grows by more than 2^8.
 #include "common.cuh"
 #include "exp2_poly.h"
@@ -64,8 +65,8 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kLaunchRegs = 168;
 template <int D, int BKV>
 struct RegSplit {
-    static constexpr int kLow = 72;
-    static constexpr int kHigh = BKV == 64 ? 208 : 216;
+    static constexpr int kLow = 80;
+    static constexpr int kHigh = 208;
     static_assert(128 * kLow + 256 * kHigh <= kThreads * kLaunchRegs, "register split exceeds the launch budget");
 };
 
@@ -87,7 +88,7 @@ struct AttnLayout {
     static constexpr int bQFull = 0, bQEmpty = 2, bKFull = 4, bKEmpty = bKFull + kNK, bVFull = bKEmpty + kNK,
                          bVEmpty = bVFull + kNV, bSFull = bVEmpty + kNV, bSFree = bSFull + 2, bPFull = bSFree + 1,
                          bPFree = bPFull + 2, bOFull = bPFree + 2, bOEmpty = bOFull + 2, bDrain = bOEmpty + 2,
-                         kNumBars = bDrain + 1;
+                         kNumBars = bDrain + 2;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 64;
     static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
@@ -142,7 +143,7 @@ struct TileCursor {
     __device__ __forceinline__ void advance(const Geo &g, const Unit &U)
     {
         if (g.nsub == 2 && s == 0) {
-            const int jt = block(U) / (g.nbh * g.nbw);
+            const int jt = (int)fdiv((uint32_t)block(U), g.fd_hw);
             if (jt * g.bt + g.subt < g.T) {
                 s = 1;
                 return;
@@ -303,7 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 TileCursor cur;
                 for (int k = 0; k < U.nkv && ok; ++k) {
                     const int j = cur.block(U);
-                    const int jt = j / (g.nbh * g.nbw), jy = (j / g.nbw) % g.nbh, jx = j % g.nbw;
+                    int jt, jy, jx;
+                    block_coords(g, j, jt, jy, jx);
                     const int tt0 = jt * g.bt + cur.s * g.subt;
                     const int ks = kc % kNK;
                     if (kc >= kNK && !mbar_wait(bar(L::bKEmpty + ks), ((kc / kNK) - 1) & 1, abort_flag)) {
@@ -343,108 +345,100 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp == 1) {
-        // ================= MMA issuer =================
+        // ================= QK issuer =================
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(128, BKV, false);
-            constexpr uint32_t idesc_pv = idesc_bf16(128, D, true);
             // descriptors of the first slab of each region; every other operand
             // is a fixed byte offset from it (added to the start-address field)
             const uint64_t q_desc = sdesc_sw128(sbase + L::kQ, 16, 1024);
             const uint64_t k_desc = sdesc_sw128(sbase + L::kK, 16, 1024);
-            const uint64_t v_desc = sdesc_sw128(sbase + L::kV, L::kKVSlab, 1024);
-            int kc = 0, vc = 0, qk_count = 0;
-            uint32_t ph_q = 0, ph_p = 0, ph_oe = 0, o_pend = 0;
+            int kc = 0, qk_count = 0;
+            uint32_t ph_q = 0;
             bool ok = true;
-            // S = Q_h K^T over D in K=16 steps; Q and K slabs are K-major, 128B swizzle
-            auto issue_qk = [&](int h, int ks) {
-                const uint64_t qa = q_desc + (uint64_t)((h * L::kDH * L::kQSlab) >> 4);
-                const uint64_t kb = k_desc + (uint64_t)((ks * L::kDH * L::kKVSlab) >> 4);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off_a = ((kk >> 2) * L::kQSlab + (kk & 3) * 32) >> 4;
-                    const uint32_t off_b = ((kk >> 2) * L::kKVSlab + (kk & 3) * 32) >> 4;
-                    umma_ss(tmem + L::kTmS, qa + off_a, kb + off_b, idesc_qk, kk > 0 ? 1u : 0u);
-                }
-            };
-            // O_h (+)= P_h V over the sub-tile in K=16 steps; P_h from TMEM, V MN-major
-            auto issue_pv = [&](int h, int vs, bool accumulate) {
-                const uint64_t vb = v_desc + (uint64_t)((vs * L::kDH * L::kKVSlab) >> 4);
-                const uint32_t d_tmem = tmem + L::tm_o(h), a_tmem = tmem + L::tm_p(h);
-#pragma unroll
-                for (int kk = 0; kk < BKV / 16; ++kk)
-                    umma_ts(d_tmem, a_tmem + kk * 8, vb + (uint64_t)((kk * 16 * 128) >> 4), idesc_pv,
-                            (accumulate || kk > 0) ? 1u : 0u);
-            };
-            auto wait_half = [&](int base, uint32_t &ph, int h) -> bool {
-                const bool r = mbar_wait(bar(base + h), (ph >> h) & 1u, abort_flag);
-                ph ^= 1u << h;
-                return r;
-            };
-            // S is shared: a QK may only overwrite it once the previous S has been
-            // copied out by its softmax warpgroup
-            auto qk = [&](int h, int ks) -> bool {
-                if (qk_count > 0 && !mbar_wait(bar(L::bSFree), (qk_count - 1) & 1, abort_flag)) return false;
-                tc_fence_after();
-                issue_qk(h, ks);
-                umma_commit(bar(L::bSFull + h));
-                ++qk_count;
-                return true;
-            };
             int u;
             for (long long idx = 0; ok && seq.get(idx, u); ++idx) {
                 const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
-                for (int h = 0; h < U.nh && ok; ++h) ok = wait_half(L::bQFull, ph_q, h);
-                if (!ok) break;
-                int ks = kc % kNK;
-                if (!mbar_wait(bar(L::bKFull + ks), (kc / kNK) & 1, abort_flag)) break;
                 for (int h = 0; h < U.nh && ok; ++h) {
-                    ok = qk(h, ks);
-                    if (ok && U.nkv == 1) umma_commit(bar(L::bQEmpty + h));
+                    ok = mbar_wait(bar(L::bQFull + h), (ph_q >> h) & 1u, abort_flag);
+                    ph_q ^= 1u << h;
                 }
-                if (!ok) break;
-                umma_commit(bar(L::bKEmpty + ks));
-                ++kc;
-                // per sub-tile k: PV_0(k), QK_0(k+1), PV_1(k), QK_1(k+1)
                 for (int k = 0; k < U.nkv && ok; ++k) {
-                    const bool next = k + 1 < U.nkv;
-                    const int vs = vc % kNV;
-                    if (!mbar_wait(bar(L::bVFull + vs), (vc / kNV) & 1, abort_flag)) { ok = false; break; }
-                    ks = kc % kNK;
-                    for (int h = 0; h < U.nh && ok; ++h) {
-                        const bool last_h = h == U.nh - 1;
-                        ok = wait_half(L::bPFull, ph_p, h);
-                        if (ok && k == 0 && ((o_pend >> h) & 1u)) {  // previous unit's epilogue read O_h
-                            ok = wait_half(L::bOEmpty, ph_oe, h);
-                            o_pend &= ~(1u << h);
+                    const int ks = kc % kNK;
+                    if (!mbar_wait(bar(L::bKFull + ks), (kc / kNK) & 1, abort_flag)) { ok = false; break; }
+                    const uint64_t kb = k_desc + (uint64_t)((ks * L::kDH * L::kKVSlab) >> 4);
+                    for (int h = 0; h < U.nh; ++h) {
+                        // S is shared: overwrite it only once the previous S has been
+                        // copied into registers by its softmax warpgroup
+                        if (qk_count > 0 && !mbar_wait(bar(L::bSFree), (qk_count - 1) & 1, abort_flag)) {
+                            ok = false;
+                            break;
                         }
-                        if (!ok) break;
                         tc_fence_after();
-                        issue_pv(h, vs, k > 0);
-                        umma_commit(bar(L::bPFree + h));
-                        if (!next) {
-                            umma_commit(bar(L::bOFull + h));
-                            o_pend |= 1u << h;
+                        const uint64_t qa = q_desc + (uint64_t)((h * L::kDH * L::kQSlab) >> 4);
+                        // S = Q_h K^T over D in K=16 steps; Q and K slabs are K-major, 128B swizzle
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t off_a = ((kk >> 2) * L::kQSlab + (kk & 3) * 32) >> 4;
+                            const uint32_t off_b = ((kk >> 2) * L::kKVSlab + (kk & 3) * 32) >> 4;
+                            umma_ss(tmem + L::kTmS, qa + off_a, kb + off_b, idesc_qk, kk > 0 ? 1u : 0u);
                         }
-                        if (last_h) umma_commit(bar(L::bVEmpty + vs));
-                        if (next) {
-                            if (h == 0 && !mbar_wait(bar(L::bKFull + ks), (kc / kNK) & 1, abort_flag)) {
-                                ok = false;
-                                break;
-                            }
-                            ok = qk(h, ks);
-                            if (!ok) break;
-                            if (k + 2 == U.nkv) umma_commit(bar(L::bQEmpty + h));
-                            if (last_h) umma_commit(bar(L::bKEmpty + ks));
-                        }
+                        umma_commit(bar(L::bSFull + h));
+                        ++qk_count;
+                        if (k == U.nkv - 1) umma_commit(bar(L::bQEmpty + h));
                     }
                     if (!ok) break;
-                    ++vc;
-                    if (next) ++kc;
+                    umma_commit(bar(L::bKEmpty + ks));
+                    ++kc;
                 }
             }
             // every MMA issued must finish before TMEM is released
             umma_commit(bar(L::bDrain));
             mbar_wait_for(bar(L::bDrain), 0, 100000000ull);
+        }
+    } else if (warp == 2) {
+        // ================= PV issuer =================
+        if (lane == 0) {
+            constexpr uint32_t idesc_pv = idesc_bf16(128, D, true);
+            const uint64_t v_desc = sdesc_sw128(sbase + L::kV, L::kKVSlab, 1024);
+            int vc = 0;
+            uint32_t ph_p = 0, ph_oe = 0, o_pend = 0;
+            bool ok = true;
+            int u;
+            for (long long idx = 0; ok && seq.get(idx, u); ++idx) {
+                const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
+                for (int k = 0; k < U.nkv && ok; ++k) {
+                    const int vs = vc % kNV;
+                    if (!mbar_wait(bar(L::bVFull + vs), (vc / kNV) & 1, abort_flag)) { ok = false; break; }
+                    const uint64_t vb = v_desc + (uint64_t)((vs * L::kDH * L::kKVSlab) >> 4);
+                    for (int h = 0; h < U.nh; ++h) {
+                        ok = mbar_wait(bar(L::bPFull + h), (ph_p >> h) & 1u, abort_flag);
+                        ph_p ^= 1u << h;
+                        if (ok && k == 0 && ((o_pend >> h) & 1u)) {  // previous unit's epilogue read O_h
+                            ok = mbar_wait(bar(L::bOEmpty + h), (ph_oe >> h) & 1u, abort_flag);
+                            ph_oe ^= 1u << h;
+                            o_pend &= ~(1u << h);
+                        }
+                        if (!ok) break;
+                        tc_fence_after();
+                        // O_h (+)= P_h V over the sub-tile in K=16 steps; P_h from TMEM, V MN-major
+                        const uint32_t d_tmem = tmem + L::tm_o(h), a_tmem = tmem + L::tm_p(h);
+#pragma unroll
+                        for (int kk = 0; kk < BKV / 16; ++kk)
+                            umma_ts(d_tmem, a_tmem + kk * 8, vb + (uint64_t)((kk * 16 * 128) >> 4), idesc_pv,
+                                    (k > 0 || kk > 0) ? 1u : 0u);
+                        umma_commit(bar(L::bPFree + h));
+                        if (k == U.nkv - 1) {
+                            umma_commit(bar(L::bOFull + h));
+                            o_pend |= 1u << h;
+                        }
+                    }
+                    if (!ok) break;
+                    umma_commit(bar(L::bVEmpty + vs));
+                    ++vc;
+                }
+            }
+            umma_commit(bar(L::bDrain + 1));
+            mbar_wait_for(bar(L::bDrain + 1), 0, 100000000ull);
         }
     } else if (warp >= 4) {
         // ================= softmax + epilogue =================
@@ -473,7 +467,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int k = 0; k < U.nkv; ++k) {
                 // the list entry after this one is loaded now and used next iteration
                 const int j_next = (U.list && e + 1 < U.cnt) ? __ldg(U.list + e + 1) : e + 1;
-                const int jt = j / (g.nbh * g.nbw), jy = (j / g.nbw) % g.nbh, jx = j % g.nbw;
+                int jt, jy, jx;
+                block_coords(g, j, jt, jy, jx);
                 const int wv = min(g.bw, g.W - jx * g.bw), hv = min(g.bh, g.Hg - jy * g.bh);
                 const int tv = min(g.subt, g.T - (jt * g.bt + s_sub * g.subt));
                 const bool full = (wv == g.bw) && (hv == g.bh) && (tv == g.subt);

@@ -13,6 +13,27 @@
 
 namespace fvattn {
 
+// Division by a run-time invariant divisor d >= 1 with a multiply and a shift
+// (Granlund and Montgomery, "Division by invariant integers using
+// multiplication", 1994, round-up variant): with l = ceil(log2 d) and
+// m = floor(2^32 (2^l - d) / d) + 1, n / d = (umulhi(n, m) + n) >> l for every
+// 0 <= n < 2^31 (the sum then stays below 2^32).
+struct FastDiv {
+    uint32_t d, m, l;
+};
+
+inline FastDiv make_fastdiv(uint32_t d)
+{
+    uint32_t l = 0;
+    while ((1ull << l) < d) ++l;
+    const uint64_t m = ((((1ull << l) - d) << 32) / d) + 1;
+    return FastDiv{d, (uint32_t)m, l};
+}
+
+#ifdef __CUDACC__
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv &f) { return (__umulhi(n, f.m) + n) >> f.l; }
+#endif
+
 // Problem geometry, resolved on the host and passed by value to every kernel.
 struct Geo {
     int B, H, N, D;
@@ -25,7 +46,20 @@ struct Geo {
     int nsub;              // sub-tiles per block along t (2 or 1)
     int rows;              // rows per sub-tile (128 or 64)
     float scale;           // softmax scale
+    FastDiv fd_nbw;        // divide by nbw
+    FastDiv fd_hw;         // divide by nbh * nbw
 };
+
+// Block j -> (jt, jy, jx) without hardware division.
+#ifdef __CUDACC__
+__device__ __forceinline__ void block_coords(const Geo &g, int j, int &jt, int &jy, int &jx)
+{
+    jt = (int)fdiv((uint32_t)j, g.fd_hw);
+    const int rem = j - jt * (int)g.fd_hw.d;
+    jy = (int)fdiv((uint32_t)rem, g.fd_nbw);
+    jx = rem - jy * g.nbw;
+}
+#endif
 
 constexpr uint32_t kFlagNonfinite = 0x1u;
 constexpr uint32_t kFlagTimeout = 0x2u;
