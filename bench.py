@@ -276,8 +276,9 @@ def run_reference(args, wl, world, rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_desc(wl)},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"per step: {desc.replace('(' + f'{t_route_full:.2f}', '(')}; "
-                                   f"routing of the full workload took {t_route_full:.2f} s once"},
+                         "sample": f"each step: attention of seeded-random whole units for ~{per_step:.1f} s "
+                                   f"(last step: {done} units) plus the full routing ({t_route_full:.2f} s, "
+                                   f"run once) counted pro rata; kept-block TFLOPS"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
