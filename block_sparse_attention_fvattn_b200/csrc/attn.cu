@@ -523,32 +523,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                         l *= alpha;
                     }
                 }
-                // P_h and O_h are free once the PV of this half's previous sub-tile is done
-                if (pw > 0 && !mbar_wait(bar(L::bPFree + h), (pw - 1) & 1, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                // p = 2^(x*scale*log2e - m); packed fp32x2 FMA/ADD, MUFU ex2 or the
-                // polynomial, bf16 pairs into P_h
+                // p = 2^(x*scale*log2e - m): packed fp32x2 FMA/ADD, MUFU ex2 (or the
+                // polynomial), packed to bf16 pairs in registers first, so this work
+                // overlaps the PV that still reads the previous P_h
                 const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m, -m);
                 uint64_t s4[4] = {0ull, 0ull, 0ull, 0ull};
+                uint32_t pk[BKV / 2];
 #pragma unroll
-                for (int c = 0; c < BKV / 32; ++c) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int q2 = 0; q2 < 16; ++q2) {
-                        const uint64_t a = f2_fma(f2_pack(x[c * 32 + 2 * q2], x[c * 32 + 2 * q2 + 1]), sl2x2, negm2);
-                        float p0, p1;
-                        if ((q2 & 7) < FV_POLY_PAIRS / 2) {
-                            exp2_poly_x2(a, p0, p1);
-                        } else {
-                            float a0, a1;
-                            f2_unpack(a, a0, a1);
-                            p0 = ex2_approx(a0);
-                            p1 = ex2_approx(a1);
-                        }
-                        s4[q2 & 3] = f2_add(s4[q2 & 3], f2_pack(p0, p1));
-                        pk[q2] = pack_bf16x2(p0, p1);
+                for (int q2 = 0; q2 < BKV / 2; ++q2) {
+                    const uint64_t a = f2_fma(f2_pack(x[2 * q2], x[2 * q2 + 1]), sl2x2, negm2);
+                    float p0, p1;
+                    if ((q2 & 7) < FV_POLY_PAIRS / 2) {
+                        exp2_poly_x2(a, p0, p1);
+                    } else {
+                        float a0, a1;
+                        f2_unpack(a, a0, a1);
+                        p0 = ex2_approx(a0);
+                        p1 = ex2_approx(a1);
                     }
-                    tmem_st16(tP + c * 16, pk);
+                    s4[q2 & 3] = f2_add(s4[q2 & 3], f2_pack(p0, p1));
+                    pk[q2] = pack_bf16x2(p0, p1);
                 }
                 float sum;
                 {
@@ -557,6 +551,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     f2_unpack(t, t0, t1);
                     sum = t0 + t1;
                 }
+                // P_h and O_h are free once the PV of this half's previous sub-tile is done
+                if (pw > 0 && !mbar_wait(bar(L::bPFree + h), (pw - 1) & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < BKV / 32; ++c) tmem_st16(tP + c * 16, pk + c * 16);
                 if (rescale) {
                     // O_h holds the sum up to the previous sub-tile (its PV is done);
                     // bring it to the new row maximum
