@@ -56,6 +56,7 @@ namespace fvattn {
 
 constexpr int kNK = 2;  // K ring stages
 constexpr int kNV = 3;  // V ring stages
+constexpr int kUnitSlots = 4;  // ring of unit ids handed from the producer to the other roles
 constexpr int kThreads = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Register split between warpgroups (setmaxnreg). The kernel is launched with
@@ -83,12 +84,15 @@ struct AttnLayout {
     // per-axis column masks: entry v-1 of each axis keeps the columns whose
     // coordinate along that axis is < v; blk_w + blk_h + sub_t <= kMaskEntries
     static constexpr int kMaskEntries = 40;
-    static constexpr int kBar = kMask + kMaskEntries * kMaskWords * 4;
+    static constexpr int kUnit = kMask + kMaskEntries * kMaskWords * 4;  // int32 unit ids
+    static constexpr int kBar = kUnit + 8 * ((kUnitSlots * 4 + 7) / 8);
     // barrier indices
     static constexpr int bQFull = 0, bQEmpty = 2, bKFull = 4, bKEmpty = bKFull + kNK, bVFull = bKEmpty + kNK,
                          bVEmpty = bVFull + kNV, bSFull = bVEmpty + kNV, bSFree = bSFull + 2, bPFull = bSFree + 1,
                          bPFree = bPFull + 2, bOFull = bPFree + 2, bOEmpty = bOFull + 2, bDrain = bOEmpty + 2,
-                         kNumBars = bDrain + 2;
+                         bUFull = bDrain + 2, bUEmpty = bUFull + kUnitSlots, kNumBars = bUEmpty + kUnitSlots;
+    // arrivals that free a unit slot: QK issuer, PV issuer and the 8 softmax warps
+    static constexpr int kUnitConsumers = 10;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 64;
     static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
@@ -154,23 +158,33 @@ struct TileCursor {
     }
 };
 
-// Units of CTA c: either its slice of the scheduled work list, or (no list)
-// the round-robin sequence c, c + C, c + 2C, ...
-struct UnitSeq {
-    const int32_t *work;
-    long long begin, end;
-    long long stride, total;
-    __device__ __forceinline__ bool get(long long idx, int &u) const
+// Rank r of the longest-first order -> unit id. The scheduler deals ranks to
+// C = gridDim.x lists in zigzag rounds (rank r sits at position r / C of list
+// zigzag(r)); without a schedule the rank is the unit id itself.
+__device__ __forceinline__ int rank_to_unit(long long r, const int32_t *work, const int32_t *cta_range)
+{
+    if (!work) return (int)r;
+    const long long C = gridDim.x;
+    const long long pos = r / C, p = r - pos * C;
+    const long long c = (pos & 1) ? C - 1 - p : p;
+    return __ldg(work + __ldg(cta_range + c) + pos);
+}
+
+// Consumer side of the unit ring: wait for the n-th slot and read its unit id
+// (-1 ends the sequence). The caller frees the slot once it has read it.
+struct UnitFeed {
+    uint32_t full0;
+    const volatile int32_t *slots;
+    int n;
+    __device__ __forceinline__ int next(volatile int *abort_flag, bool &ok, int &slot)
     {
-        if (work) {
-            if (begin + idx >= end) return false;
-            u = __ldg(work + begin + idx);
-            return true;
+        slot = n % kUnitSlots;
+        if (!mbar_wait(full0 + 8u * (uint32_t)slot, (uint32_t)(n / kUnitSlots) & 1u, abort_flag)) {
+            ok = false;
+            return -1;
         }
-        const long long v = begin + idx * stride;
-        if (v >= total) return false;
-        u = (int)v;
-        return true;
+        ++n;
+        return slots[slot];
     }
 };
 
@@ -246,6 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t cnt = 1;
             if (b == L::bSFree || b == L::bPFull || b == L::bPFull + 1 || b == L::bOEmpty || b == L::bOEmpty + 1)
                 cnt = 128;  // arrived on by all 128 threads of a softmax warpgroup
+            if (b >= L::bUEmpty && b < L::bUEmpty + kUnitSlots) cnt = L::kUnitConsumers;
             mbar_init(bar(b), cnt);
         }
         fence_mbar_init();
@@ -259,17 +274,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    UnitSeq seq;
-    seq.work = work;
-    if (work) {
-        seq.begin = __ldg(cta_range + blockIdx.x);
-        seq.end = __ldg(cta_range + blockIdx.x + 1);
-    } else {
-        seq.begin = blockIdx.x;
-        seq.end = 0;
-    }
-    seq.stride = gridDim.x;
-    seq.total = (long long)g.BH * g.nb;
+    // Units are taken dynamically, longest first, from a counter shared by all
+    // CTAs (workspace header word 1); the producer thread takes them and hands
+    // them to the other roles through the unit ring.
+    const long long n_units = (long long)g.BH * g.nb;
+    uint32_t *unit_cursor = status + 1, *ctas_done = status + 2;
+    volatile int32_t *unit_slots = reinterpret_cast<volatile int32_t *>(gbase + L::kUnit);
+    UnitFeed feed{bar(L::bUFull), unit_slots, 0};
 
     constexpr uint32_t kTileBytes = (uint32_t)L::kDH * BKV * 128u;
     const uint32_t q_bytes = (uint32_t)L::kDH * (uint32_t)g.rows * 128u;
@@ -284,8 +295,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             int kc = 0, vc = 0;
             uint32_t q_par = 0, q_used = 0;  // per half: loads issued & 1, any load issued
             bool ok = true;
-            int u;
-            for (long long idx = 0; ok && seq.get(idx, u); ++idx) {
+            for (int n = 0; ok; ++n) {
+                const int slot = n % kUnitSlots;
+                if (n >= kUnitSlots &&
+                    !mbar_wait(bar(L::bUEmpty + slot), (uint32_t)((n / kUnitSlots) - 1) & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const long long r = (long long)atomicAdd(unit_cursor, 1u);
+                const int u = r < n_units ? rank_to_unit(r, work, cta_range) : -1;
+                unit_slots[slot] = u;
+                mbar_arrive(bar(L::bUFull + slot));  // release: the id is visible to the waiting roles
+                if (u < 0) break;
                 const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
                 const int x0 = U.ix * g.bw, y0 = U.iy * g.bh, t0 = U.it * g.bt;
                 for (int h = 0; h < U.nh && ok; ++h) {
@@ -355,8 +376,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             int kc = 0, qk_count = 0;
             uint32_t ph_q = 0;
             bool ok = true;
-            int u;
-            for (long long idx = 0; ok && seq.get(idx, u); ++idx) {
+            while (ok) {
+                int slot;
+                const int u = feed.next(abort_flag, ok, slot);
+                if (!ok) break;
+                mbar_arrive(bar(L::bUEmpty + slot));
+                if (u < 0) break;
                 const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
                 for (int h = 0; h < U.nh && ok; ++h) {
                     ok = mbar_wait(bar(L::bQFull + h), (ph_q >> h) & 1u, abort_flag);
@@ -403,8 +428,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             int vc = 0;
             uint32_t ph_p = 0, ph_oe = 0, o_pend = 0;
             bool ok = true;
-            int u;
-            for (long long idx = 0; ok && seq.get(idx, u); ++idx) {
+            while (ok) {
+                int slot;
+                const int u = feed.next(abort_flag, ok, slot);
+                if (!ok) break;
+                mbar_arrive(bar(L::bUEmpty + slot));
+                if (u < 0) break;
                 const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
                 for (int k = 0; k < U.nkv && ok; ++k) {
                     const int vs = vc % kNV;
@@ -455,8 +484,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r_t = row / (g.bh * g.bw), r_y = (row / g.bw) % g.bh, r_x = row % g.bw;
         int sf = 0, of = 0, pw = 0;  // S tiles received, O tiles received, P tiles written
         bool ok = true;
-        int u;
-        for (long long idx = 0; ok && seq.get(idx, u); ++idx) {
+        while (ok) {
+            int slot;
+            const int u = feed.next(abort_flag, ok, slot);
+            if (!ok) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(L::bUEmpty + slot));  // every lane has read the id
+            if (u < 0) break;
             const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
             if (h >= U.nh) continue;
             const int qt = U.it * g.bt + h * g.subt + r_t, qy = U.iy * g.bh + r_y, qx = U.ix * g.bw + r_x;
@@ -620,6 +654,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         if (*abort_flag) atomicOr(status, kFlagTimeout);
         if (cta_ns) cta_ns[blockIdx.x] = (int64_t)(globaltimer_ns() - t_start);
+        // every CTA has taken its last rank before it gets here; the last CTA to
+        // finish resets the shared counters for the next launch on this workspace
+        __threadfence();
+        if (atomicAdd(ctas_done, 1u) == gridDim.x - 1) {
+            atomicExch(unit_cursor, 0u);
+            atomicExch(ctas_done, 0u);
+        }
     }
 }
 

@@ -146,6 +146,9 @@ FVATTN_API fvattn_status fvattn_route(const fvattn_problem *prob, const void *q,
  * zigzag(r) = r mod 2C < C ? r mod C : 2C-1 - r mod C, so each round of C
  * consecutive ranks (one head's units run together, which keeps its key/value
  * blocks in L2) gives every CTA one unit, alternating the largest end.
+ * cta_cost is the cost of that static deal; fvattn_sparse_attn runs the same
+ * ranked order dynamically (see there), which evens out what the cost model
+ * misses.
  *
  *   kv_cnt, kv_idx  the lists from fvattn_route (ignored if dense != 0)
  *   dense           nonzero: schedule the all-blocks problem
@@ -174,6 +177,11 @@ FVATTN_API fvattn_status fvattn_schedule(const fvattn_problem *prob, const int32
  *   q, k, v        bf16 [B,H,N,D]
  *   kv_cnt, kv_idx lists from fvattn_route (ignored if dense)
  *   work, cta_range from fvattn_schedule with the same num_ctas and dense flag
+ *                  (both NULL: units in index order). The CTAs take ranks
+ *                  0, 1, 2, ... of the scheduler's longest-first order from a
+ *                  counter shared through the workspace (rank r is entry
+ *                  r / num_ctas of list zigzag(r)), so a CTA that finishes early
+ *                  takes the next unit; the last CTA resets the counter.
  *   num_ctas       grid size (0 = SM count); must match fvattn_schedule's
  *   out            bf16 [B,H,N,D]; every valid token is written
  *   cta_ns         out int64 [num_ctas] busy time of each CTA in ns, or NULL
