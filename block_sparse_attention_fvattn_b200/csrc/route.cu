@@ -22,90 +22,150 @@ namespace fvattn {
 
 // ---------------------------------------------------------------------------
 // K1
-template <int D>
-__global__ void __launch_bounds__(256) pool_kernel(Geo g, const __nv_bfloat16 *__restrict__ q,
-                                                   const __nv_bfloat16 *__restrict__ k, float *__restrict__ qbar,
-                                                   float *__restrict__ kbarT)
+// A CTA pools a strip of blocks: one block row (jt, jy) and a run of block
+// columns [jx0, jx1). For every (t, y) the strip's tokens x0 .. x1-1 are one
+// contiguous run of (x1 - x0) * D bf16 values, so the CTA streams tv * yv
+// contiguous runs. Thread tid owns the 16-byte positions tid + kPoolThreads*s
+// of every run (s < NS): a fixed token column and d-chunk, so each load is a
+// pointer step and the running sums stay in registers (packed fp32x2 adds).
+// At the end the columns of each block are added in ascending x through
+// shared memory.
+constexpr int kPoolThreads = 256;
+
+struct PoolPlan {
+    int nxs;  // strips per block row
+    int ns;   // positions per thread and run (1, 2, 3, 4 or 8)
+};
+
+__host__ __device__ inline PoolPlan pool_plan(int nbw, int bw, int D)
 {
-    constexpr int LPT = D / 8;  // lanes per token (one 16-byte chunk each)
-    constexpr int kBatch = 8;   // loads in flight per lane
-    const int lane = threadIdx.x & 31;
-    const long long warp = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    const long long per = (long long)g.BH * g.nb;
-    if (warp >= 2 * per) return;
-    const int which = warp >= per ? 1 : 0;
-    const long long rem = warp - which * per;
-    const int bh = (int)(rem / g.nb), j = (int)(rem - (long long)bh * g.nb);
-    const int jt = j / (g.nbh * g.nbw), jy = (j / g.nbw) % g.nbh, jx = j % g.nbw;
-    const int t0 = jt * g.bt, y0 = jy * g.bh, x0 = jx * g.bw;
-    const int tv = min(g.bt, g.T - t0), yv = min(g.bh, g.Hg - y0), xv = min(g.bw, g.W - x0);
+    const int lpt = D / 8;
+    const int cap = kPoolThreads * 3 / (bw * lpt);  // block columns per strip at NS <= 3
+    PoolPlan pl;
+    pl.nxs = cap >= 1 ? (nbw + cap - 1) / cap : nbw;
+    const int xb = (nbw + pl.nxs - 1) / pl.nxs;
+    const int need = (xb * bw * lpt + kPoolThreads - 1) / kPoolThreads;
+    pl.ns = need <= 4 ? need : 8;
+    return pl;
+}
+
+template <int D, int NS>
+__global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geo g, int nxs, const __nv_bfloat16 *__restrict__ q,
+                                                            const __nv_bfloat16 *__restrict__ k,
+                                                            float *__restrict__ qbar, float *__restrict__ kbarT)
+{
+    constexpr int LPT = D / 8;  // 16-byte chunks per token
+    constexpr int RB = NS >= 8 ? 1 : 8 / NS;  // runs per batch of loads
+    extern __shared__ __align__(16) float red[];  // [positions][8]
+
+    // task -> (which, bh, jt, jy, xs); xs fastest so neighbouring CTAs read
+    // neighbouring memory
+    long long task = blockIdx.x;
+    const int xs = (int)(task % nxs);
+    task /= nxs;
+    const int nbt = g.nbt, nbh = g.nbh, nbw = g.nbw;
+    const int jy = (int)(task % nbh);
+    task /= nbh;
+    const int jt = (int)(task % nbt);
+    task /= nbt;
+    const long long per = g.BH;
+    const int which = task >= per ? 1 : 0;
+    const int bh = (int)(task - which * per);
+
+    const int jx0 = (int)((long long)xs * nbw / nxs), jx1 = (int)((long long)(xs + 1) * nbw / nxs);
+    const int x0 = jx0 * g.bw, x1 = min(jx1 * g.bw, g.W);
+    const int t0 = jt * g.bt, y0 = jy * g.bh;
+    const int tv = min(g.bt, g.T - t0), yv = min(g.bh, g.Hg - y0);
+    const int npos = (x1 - x0) * LPT;
+    const int tid = threadIdx.x;
+
     const __nv_bfloat16 *src = which ? k : q;
-    const uint4 *base = reinterpret_cast<const uint4 *>(src + (size_t)bh * g.N * D);
-    const int cpr = xv * LPT;  // 16-byte chunks in one (t, y) run of xv tokens
+    const uint4 *run = reinterpret_cast<const uint4 *>(src + (size_t)bh * g.N * D) +
+                       (((size_t)t0 * g.Hg + y0) * g.W + x0) * LPT;
+    const size_t run_step = (size_t)g.W * LPT;                            // next y
+    const size_t t_step = ((size_t)g.Hg - (size_t)yv) * g.W * LPT;         // extra at a new t
 
-    float acc[8];
+    bool own[NS];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    for (int s = 0; s < NS; ++s) own[s] = tid + kPoolThreads * s < npos;
+    uint64_t acc[NS][4];
+#pragma unroll
+    for (int s = 0; s < NS; ++s)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[s][c] = 0ull;
 
-    // cursor over (t, y, chunk) in the order t, y, chunk; each lane starts at
-    // chunk `lane` and advances by 32 chunks. Its d-chunk (lane % LPT) is fixed.
-    int t = t0, y = y0, e = lane;
-    while (e >= cpr && t < t0 + tv) {
-        e -= cpr;
-        if (++y == y0 + yv) { y = y0; ++t; }
-    }
-    while (t < t0 + tv) {
-        uint4 v[kBatch];
-        bool ok[kBatch];
+    const int nrun = tv * yv;
+    int y = 0;
+    for (int r = 0; r < nrun; r += RB) {
+        uint4 v[RB][NS];
 #pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            ok[b] = t < t0 + tv;
-            if (ok[b]) {
-                const size_t tok = ((size_t)t * g.Hg + y) * g.W + x0;
-                v[b] = __ldg(base + tok * LPT + e);
-                e += 32;
-                while (e >= cpr && t < t0 + tv) {
-                    e -= cpr;
-                    if (++y == y0 + yv) { y = y0; ++t; }
+        for (int b = 0; b < RB; ++b) {
+            const bool ok = r + b < nrun;
+#pragma unroll
+            for (int s = 0; s < NS; ++s)
+                if (ok && own[s]) v[b][s] = __ldg(run + tid + kPoolThreads * s);
+            if (ok) {
+                run += run_step;
+                if (++y == yv) {
+                    y = 0;
+                    run += t_step;
                 }
             }
         }
 #pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            if (ok[b]) {
-                const uint32_t w[4] = {v[b].x, v[b].y, v[b].z, v[b].w};
+        for (int b = 0; b < RB; ++b) {
+            if (r + b < nrun) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    acc[2 * c] += __uint_as_float(w[c] << 16);
-                    acc[2 * c + 1] += __uint_as_float(w[c] & 0xFFFF0000u);
+                for (int s = 0; s < NS; ++s) {
+                    if (own[s]) {
+                        const uint32_t w[4] = {v[b][s].x, v[b][s].y, v[b][s].z, v[b][s].w};
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            acc[s][c] = f2_add(acc[s][c], f2_pack(__uint_as_float(w[c] << 16),
+                                                                  __uint_as_float(w[c] & 0xFFFF0000u)));
+                    }
                 }
             }
         }
     }
-    // lanes with the same d-chunk combine in a fixed order
+    // every load of this CTA has been consumed: the selection kernel, if it
+    // was launched as a programmatic dependent, may begin its launch
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
 #pragma unroll
-    for (int off = LPT; off < 32; off <<= 1) {
+    for (int s = 0; s < NS; ++s) {
+        if (own[s]) {
+            float4 *o = reinterpret_cast<float4 *>(red + (size_t)(tid + kPoolThreads * s) * 8);
+            float a[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] += __shfl_xor_sync(0xFFFFFFFFu, acc[c], off);
-    }
-    if (lane < LPT) {
-        const float inv = 1.0f / (float)(tv * yv * xv);
-        const int d0 = lane * 8;
-        if (!which) {
-            float4 *o = reinterpret_cast<float4 *>(qbar + ((size_t)bh * g.nb + j) * D + d0);
-            o[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-            o[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
-        } else {
-            float *o = kbarT + ((size_t)bh * D + d0) * g.nbp + j;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) o[(size_t)c * g.nbp] = acc[c] * inv;
+            for (int c = 0; c < 4; ++c) f2_unpack(acc[s][c], a[2 * c], a[2 * c + 1]);
+            o[0] = make_float4(a[0], a[1], a[2], a[3]);
+            o[1] = make_float4(a[4], a[5], a[6], a[7]);
         }
+    }
+    __syncthreads();
+    // output (block jx, channel d): the strip's token columns of that block in
+    // ascending x
+    const int nout = (jx1 - jx0) * D;
+    for (int o = tid; o < nout; o += kPoolThreads) {
+        const int jl = o / D, d = o - jl * D;
+        const int xa = jl * g.bw, xb = min(xa + g.bw, x1 - x0);
+        float sum = 0.f;
+        for (int x = xa; x < xb; ++x) sum += red[x * D + d];
+        const float mean = sum * (1.0f / (float)(tv * yv * (xb - xa)));
+        const int j = (jt * nbh + jy) * nbw + jx0 + jl;
+        if (!which) qbar[((size_t)bh * g.nb + j) * D + d] = mean;
+        else kbarT[((size_t)bh * D + d) * g.nbp + j] = mean;
     }
 }
 
 // ---------------------------------------------------------------------------
 // K2
 constexpr int kSelRows = 8;  // query blocks per CTA (rows of the score tile), one per warp
+// Rows of up to 256 blocks select by a warp sort of their keys; longer rows by
+// a binary search over the key space (fewer passes over the row's elements).
+template <int EPL>
+constexpr bool kSortedSelect = EPL == 1 || EPL == 2 || EPL == 4 || EPL == 8;
 
 __device__ __forceinline__ float warp_sum(float v)
 {
@@ -139,59 +199,160 @@ __device__ __forceinline__ uint32_t order_key(float s)
     const uint32_t u = __float_as_uint(s);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
-
-template <int D, int EPL>
-__global__ void __launch_bounds__(256) score_select_kernel(Geo g, const float *__restrict__ qbar,
-                                                           const float *__restrict__ kbarT, float p, int k_min,
-                                                           int32_t *__restrict__ kv_cnt, int32_t *__restrict__ kv_idx,
-                                                           float *__restrict__ probs, uint32_t *__restrict__ status)
+// Inverse of order_key on the keys of finite floats.
+__device__ __forceinline__ float key_float(uint32_t key)
 {
-    extern __shared__ __align__(16) float sel_smem[];
-    float *qsT = sel_smem;                 // [D][kSelRows]
-    float *sc = sel_smem + D * kSelRows;   // [kSelRows][nbp]
-    const int bh = blockIdx.y;
-    const int i0 = blockIdx.x * kSelRows;
-    const int nrow = min(kSelRows, g.nb - i0);
-    const int nbp = g.nbp;
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
 
-    for (int idx = threadIdx.x; idx < kSelRows * D; idx += blockDim.x) {
-        const int r = idx / D, d = idx - r * D;
-        qsT[d * kSelRows + r] = (r < nrow) ? qbar[((size_t)bh * g.nb + i0 + r) * D + d] : 0.f;
+// Bitonic sort, descending, of the 32*EPL keys a warp holds: lane l holds
+// positions l*EPL .. l*EPL+EPL-1. Exchanges between positions closer than
+// EPL stay in a lane's registers; the others go through shuffles.
+template <int EPL>
+__device__ __forceinline__ void warp_sort_desc(uint32_t (&key)[EPL], int lane)
+{
+    constexpr int N = 32 * EPL;
+#pragma unroll
+    for (int k = 2; k <= N; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            if (j < EPL) {
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) {
+                    if (e & j) continue;
+                    const int f = e | j;
+                    // the pair (e, f) is kept descending where bit k of the position is 0
+                    const bool desc = k < EPL ? ((e & k) == 0) : ((lane & (k / EPL)) == 0);
+                    const uint32_t a = key[e], b = key[f];
+                    const uint32_t hi = max(a, b), lo = min(a, b);
+                    key[e] = desc ? hi : lo;
+                    key[f] = desc ? lo : hi;
+                }
+            } else {
+                const int lm = j / EPL;  // partner lane = lane ^ lm
+                const bool lower = (lane & lm) == 0;
+                const bool desc = (lane & (k / EPL)) == 0;
+                const bool keep_max = lower == desc;
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) {
+                    const uint32_t o = __shfl_xor_sync(0xFFFFFFFFu, key[e], lm);
+                    key[e] = keep_max ? max(key[e], o) : min(key[e], o);
+                }
+            }
+        }
     }
-    __syncthreads();
+}
 
-    // ---- block scores: each thread owns 4 consecutive key blocks x kSelRows rows
-    const float *kb = kbarT + (size_t)bh * D * nbp;
-    for (int c0 = threadIdx.x * 4; c0 < nbp; c0 += blockDim.x * 4) {
-        float acc[kSelRows][4];
+// Key at sorted position r (warp-uniform) of keys sorted by warp_sort_desc.
+template <int EPL>
+__device__ __forceinline__ uint32_t key_at(const uint32_t (&key)[EPL], int r)
+{
+    const int e = r % EPL;
+    uint32_t mine = key[0];
 #pragma unroll
-        for (int r = 0; r < kSelRows; ++r)
+    for (int x = 1; x < EPL; ++x)
+        if (e == x) mine = key[x];
+    return __shfl_sync(0xFFFFFFFFu, mine, r / EPL);
+}
+
+// The d range of the score dot products is cut into S slices so that all
+// 256 threads work on small tiles: thread w owns 4 consecutive key blocks x
+// kSelRows rows over one slice (the slice's loads are all in flight at once
+// when it is short). Per element the slice sums are fp32 fmas in ascending d,
+// and the slices are then added in ascending order.
+__host__ __device__ constexpr int sel_slices(int nbp)
+{
+    return (nbp >> 2) >= 256 ? 1 : (nbp >> 2) >= 128 ? 2 : (nbp >> 2) >= 64 ? 4 : 8;
+}
+
+template <int D, int S>
+__device__ __forceinline__ void score_tile(const float *kb, const float *qsT, float *sc, int nbp, float scale)
+{
+    constexpr int DS = D / S;
+    constexpr int kUnroll = DS <= 16 ? DS : 8;
+    const int NQ = nbp >> 2;
+    for (int w = threadIdx.x; w < NQ * S; w += blockDim.x) {
+        const int sl = S == 1 ? 0 : w / NQ;
+        const int c0 = (w - sl * NQ) * 4;
+        uint64_t acc[kSelRows][2];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
-#pragma unroll 8
-        for (int d = 0; d < D; ++d) {
-            const float4 kv = __ldg(reinterpret_cast<const float4 *>(kb + (size_t)d * nbp + c0));
-            const float4 *qv = reinterpret_cast<const float4 *>(qsT + d * kSelRows);
+        for (int r = 0; r < kSelRows; ++r) acc[r][0] = acc[r][1] = 0ull;
+        const float *kp = kb + (size_t)(sl * DS) * nbp + c0;
+        const float *qp = qsT + sl * DS * kSelRows;
+#pragma unroll kUnroll
+        for (int d = 0; d < DS; ++d) {
+            const float4 kv = __ldg(reinterpret_cast<const float4 *>(kp + (size_t)d * nbp));
+            const uint64_t k01 = f2_pack(kv.x, kv.y), k23 = f2_pack(kv.z, kv.w);
+            const float4 *qv = reinterpret_cast<const float4 *>(qp + d * kSelRows);
 #pragma unroll
             for (int r4 = 0; r4 < kSelRows / 4; ++r4) {
                 const float4 qq = qv[r4];
                 const float qr[4] = {qq.x, qq.y, qq.z, qq.w};
 #pragma unroll
                 for (int rr = 0; rr < 4; ++rr) {
-                    acc[r4 * 4 + rr][0] = fmaf(qr[rr], kv.x, acc[r4 * 4 + rr][0]);
-                    acc[r4 * 4 + rr][1] = fmaf(qr[rr], kv.y, acc[r4 * 4 + rr][1]);
-                    acc[r4 * 4 + rr][2] = fmaf(qr[rr], kv.z, acc[r4 * 4 + rr][2]);
-                    acc[r4 * 4 + rr][3] = fmaf(qr[rr], kv.w, acc[r4 * 4 + rr][3]);
+                    const uint64_t q2 = f2_pack(qr[rr], qr[rr]);
+                    acc[r4 * 4 + rr][0] = f2_fma(q2, k01, acc[r4 * 4 + rr][0]);
+                    acc[r4 * 4 + rr][1] = f2_fma(q2, k23, acc[r4 * 4 + rr][1]);
                 }
             }
         }
+        float *dst = sc + (size_t)sl * kSelRows * nbp;
+        const float f = S == 1 ? scale : 1.0f;
 #pragma unroll
         for (int r = 0; r < kSelRows; ++r) {
-            float4 o = make_float4(g.scale * acc[r][0], g.scale * acc[r][1], g.scale * acc[r][2],
-                                   g.scale * acc[r][3]);
-            *reinterpret_cast<float4 *>(sc + r * nbp + c0) = o;
+            float a0, a1, a2, a3;
+            f2_unpack(acc[r][0], a0, a1);
+            f2_unpack(acc[r][1], a2, a3);
+            *reinterpret_cast<float4 *>(dst + r * nbp + c0) = make_float4(f * a0, f * a1, f * a2, f * a3);
         }
     }
+    if (S > 1) {
+        __syncthreads();
+        const int n4 = kSelRows * nbp / 4;
+        for (int x = threadIdx.x; x < n4; x += blockDim.x) {
+            float4 t = reinterpret_cast<const float4 *>(sc)[x];
+#pragma unroll
+            for (int sl = 1; sl < S; ++sl) {
+                const float4 u = reinterpret_cast<const float4 *>(sc + (size_t)sl * kSelRows * nbp)[x];
+                t.x += u.x;
+                t.y += u.y;
+                t.z += u.z;
+                t.w += u.w;
+            }
+            reinterpret_cast<float4 *>(sc)[x] = make_float4(scale * t.x, scale * t.y, scale * t.z, scale * t.w);
+        }
+    }
+}
+
+// The CTA (8 warps) routes query blocks i0 .. i0+7 of head bh: scores into
+// shared memory, then one warp per row selects and compacts. Shared memory:
+// (D + sel_slices(nbp) * nbp) * kSelRows floats.
+template <int D, int EPL>
+__device__ __forceinline__ void select_rows(const Geo &g, int bh, int i0, float *sel_smem,
+                                            const float *qbar, const float *kbarT, float p,
+                                            int k_min, int32_t *__restrict__ kv_cnt, int32_t *__restrict__ kv_idx,
+                                            float *__restrict__ probs, uint32_t *__restrict__ status)
+{
+    float *qsT = sel_smem;                 // [D][kSelRows]
+    float *sc = sel_smem + D * kSelRows;   // [S][kSelRows][nbp]; slice 0 ends up holding the scores
+    const int nrow = min(kSelRows, g.nb - i0);
+    const int nbp = g.nbp;
+
+    // launched as a programmatic dependent of the pooling kernel: wait for it
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    for (int idx = threadIdx.x; idx < kSelRows * D; idx += blockDim.x) {
+        const int r = idx / D, d = idx - r * D;
+        qsT[d * kSelRows + r] = (r < nrow) ? qbar[((size_t)bh * g.nb + i0 + r) * D + d] : 0.f;
+    }
+    __syncthreads();
+
+    // ---- block scores
+    const float *kb = kbarT + (size_t)bh * D * nbp;
+    const int S = sel_slices(nbp);
+    if (S == 8) score_tile<D, 8>(kb, qsT, sc, nbp, g.scale);
+    else if (S == 4) score_tile<D, 4>(kb, qsT, sc, nbp, g.scale);
+    else if (S == 2) score_tile<D, 2>(kb, qsT, sc, nbp, g.scale);
+    else score_tile<D, 1>(kb, qsT, sc, nbp, g.scale);
     __syncthreads();
 
     // ---- selection: one warp per row
@@ -201,21 +362,21 @@ __global__ void __launch_bounds__(256) score_select_kernel(Geo g, const float *_
     for (int r = warp; r < nrow; r += blockDim.x >> 5) {
         const int i = i0 + r;
         const size_t row = (size_t)bh * nb + i;
-        const float *srow = sc + r * nbp;
+        float *srow = sc + r * nbp;
         int32_t *out = kv_idx + row * (size_t)nb;
-        float sv[EPL];
+        uint32_t key[EPL];  // order_key of the scores; 0 (below every real key) past nb
         bool bad = false;
         float mx = -INFINITY;
 #pragma unroll
         for (int e = 0; e < EPL; ++e) {
             const int j = lane + 32 * e;
-            float s = -INFINITY;
+            key[e] = 0u;
             if (j < nb) {
-                s = srow[j] + 0.0f;  // folds -0 into +0
+                const float s = srow[j] + 0.0f;  // folds -0 into +0
                 if (!isfinite(s)) bad = true;
                 else mx = fmaxf(mx, s);
+                key[e] = order_key(s);
             }
-            sv[e] = s;
         }
         if (__any_sync(0xFFFFFFFFu, bad)) {
             // repair: a row with an unusable score keeps every block
@@ -234,128 +395,129 @@ __global__ void __launch_bounds__(256) score_select_kernel(Geo g, const float *_
             continue;
         }
         mx = warp_max(mx);
-        float pv[EPL];
-        uint32_t key[EPL];
-        float z = 0.f;
-        uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) {
-            const int j = lane + 32 * e;
-            if (j < nb) {
-                pv[e] = expf(sv[e] - mx);
-                key[e] = order_key(sv[e]);
-                kmin = min(kmin, key[e]);
-                kmax = max(kmax, key[e]);
-            } else {
-                pv[e] = 0.f;
-                key[e] = 0u;  // below every real key; never selected
-            }
-            z += pv[e];
-        }
-        z = warp_sum(z);
-        kmin = warp_min_u(kmin);
-        kmax = warp_max_u(kmax);
 
-        bool all_sel = false;
+        bool all_sel = p >= 1.0f;
         uint32_t kap = 0;   // boundary key of the kept set
         int ntie = 0;       // how many blocks with key == kap are kept (lowest indices)
-        int m = nb;
-        if (p >= 1.0f) {
-            all_sel = true;
-        } else {
-            const float target = p * z;
-            // largest key t with mass(key >= t) >= target: 4-ary search, three
-            // independent reductions per step
-            uint32_t lo = kmin, hi = kmax + 1u;
-            while (hi - lo > 1u) {
-                const uint32_t q4 = (hi - lo) >> 2;
-                const uint32_t t1 = lo + (q4 ? q4 : 1u), t2 = lo + (q4 ? 2u * q4 : 1u),
-                               t3 = lo + (q4 ? 3u * q4 : 1u);
-                float m1 = 0.f, m2 = 0.f, m3 = 0.f;
+        float z;            // softmax denominator
+        if constexpr (kSortedSelect<EPL>) {
+            // Sort the keys, then C_before(r) = mass of sorted positions < r
+            // by a prefix scan in rank order; position r is kept by Top-p
+            // while C_before(r) < p * z.
+            uint32_t sk[EPL];
 #pragma unroll
-                for (int e = 0; e < EPL; ++e) {
-                    m1 += (key[e] >= t1) ? pv[e] : 0.f;
-                    m2 += (key[e] >= t2) ? pv[e] : 0.f;
-                    m3 += (key[e] >= t3) ? pv[e] : 0.f;
-                }
-                m1 = warp_sum(m1);
-                m2 = warp_sum(m2);
-                m3 = warp_sum(m3);
-                if (m3 >= target) {
-                    lo = t3;
-                } else if (m2 >= target) {
-                    lo = t2;
-                    hi = t3;
-                } else if (m1 >= target) {
-                    lo = t1;
-                    hi = t2;
-                } else {
-                    hi = t1;
-                }
-            }
-            const uint32_t kp = lo;
-            float mass_gt = 0.f, p_eq = 0.f;
-            int cnt_gt = 0, n_eq = 0;
+            for (int e = 0; e < EPL; ++e) sk[e] = key[e];
+            warp_sort_desc<EPL>(sk, lane);
+            float c[EPL];
+            float run = 0.f;
 #pragma unroll
             for (int e = 0; e < EPL; ++e) {
-                mass_gt += (key[e] >= kp + 1u) ? pv[e] : 0.f;
-                cnt_gt += (key[e] > kp) ? 1 : 0;
-                n_eq += (key[e] == kp) ? 1 : 0;
-                if (key[e] == kp) p_eq = pv[e];
+                c[e] = run;  // mass before this position, within the lane
+                run += sk[e] ? expf(key_float(sk[e]) - mx) : 0.f;
             }
-            mass_gt = warp_sum(mass_gt);
-            cnt_gt = (int)__reduce_add_sync(0xFFFFFFFFu, (uint32_t)cnt_gt);
-            n_eq = (int)__reduce_add_sync(0xFFFFFFFFu, (uint32_t)n_eq);
-            p_eq = warp_max(p_eq);
-            // blocks tied at the boundary enter one at a time, lowest index first
-            float accm = mass_gt;
-            int n = 0;
-            while (n < n_eq && accm < target) {
-                accm += p_eq;
-                ++n;
-            }
-            const int m_p = cnt_gt + n;
-            m = max(m_p, k_min);
-            if (m >= nb) {
-                all_sel = true;
-            } else if (m == m_p) {
-                kap = kp;
-                ntie = n;
-            } else {
-                // Top-k floor binds: boundary key of rank m (4-ary search on counts)
-                uint32_t lo2 = kmin, hi2 = kp + 1u;
-                while (hi2 - lo2 > 1u) {
-                    const uint32_t q4 = (hi2 - lo2) >> 2;
-                    const uint32_t t1 = lo2 + (q4 ? q4 : 1u), t2 = lo2 + (q4 ? 2u * q4 : 1u),
-                                   t3 = lo2 + (q4 ? 3u * q4 : 1u);
-                    uint32_t c1 = 0, c2 = 0, c3 = 0;
+            float incl = run;
 #pragma unroll
-                    for (int e = 0; e < EPL; ++e) {
-                        c1 += (key[e] >= t1) ? 1u : 0u;
-                        c2 += (key[e] >= t2) ? 1u : 0u;
-                        c3 += (key[e] >= t3) ? 1u : 0u;
-                    }
-                    c1 = __reduce_add_sync(0xFFFFFFFFu, c1);
-                    c2 = __reduce_add_sync(0xFFFFFFFFu, c2);
-                    c3 = __reduce_add_sync(0xFFFFFFFFu, c3);
-                    if (c3 >= (uint32_t)m) {
-                        lo2 = t3;
-                    } else if (c2 >= (uint32_t)m) {
-                        lo2 = t2;
-                        hi2 = t3;
-                    } else if (c1 >= (uint32_t)m) {
-                        lo2 = t1;
-                        hi2 = t2;
-                    } else {
-                        hi2 = t1;
-                    }
+            for (int o = 1; o < 32; o <<= 1) {
+                const float t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            z = __shfl_sync(0xFFFFFFFFu, incl, 31);
+            float excl = __shfl_up_sync(0xFFFFFFFFu, incl, 1);
+            if (lane == 0) excl = 0.f;
+            if (!all_sel) {
+                const float target = p * z;
+                int m_p = 0;
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) m_p += __popc(__ballot_sync(0xFFFFFFFFu, excl + c[e] < target));
+                const int m = max(m_p, k_min);
+                if (m >= nb) {
+                    all_sel = true;
+                } else {
+                    kap = key_at<EPL>(sk, m - 1);
+                    int c_gt = 0;
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) c_gt += (key[e] > kap) ? 1 : 0;
+                    ntie = m - (int)__reduce_add_sync(0xFFFFFFFFu, (uint32_t)c_gt);
                 }
-                kap = lo2;
-                int c_gt = 0;
+            }
+        } else {
+            // Binary search over the key space: the largest key t whose mass
+            // mass(key >= t) reaches p * z is the Top-p boundary. The masses
+            // replace the scores in the row's shared memory.
+            uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+            float zl = 0.f;
 #pragma unroll
-                for (int e = 0; e < EPL; ++e) c_gt += (key[e] > kap) ? 1 : 0;
-                c_gt = (int)__reduce_add_sync(0xFFFFFFFFu, (uint32_t)c_gt);
-                ntie = m - c_gt;
+            for (int e = 0; e < EPL; ++e) {
+                const int j = lane + 32 * e;
+                if (j < nb) {
+                    const float pj = expf(key_float(key[e]) - mx);
+                    srow[j] = pj;
+                    kmin = min(kmin, key[e]);
+                    kmax = max(kmax, key[e]);
+                    zl += pj;
+                }
+            }
+            const float *pvr = srow;  // pv of block j at pvr[j]; read only where key[e] != 0
+            auto pv = [&](int e) { return key[e] ? pvr[lane + 32 * e] : 0.f; };
+            z = warp_sum(zl);
+            kmin = warp_min_u(kmin);
+            kmax = warp_max_u(kmax);
+            if (!all_sel) {
+                const float target = p * z;
+                uint32_t lo = kmin, hi = kmax + 1u;  // mass(>= lo) >= target > mass(>= hi)
+                while (hi - lo > 1u) {
+                    const uint32_t mid = lo + ((hi - lo) >> 1);
+                    float mm = 0.f;
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) mm += (key[e] >= mid) ? pv(e) : 0.f;
+                    if (warp_sum(mm) >= target) lo = mid;
+                    else hi = mid;
+                }
+                const uint32_t kp = lo;
+                float mass_gt = 0.f, p_eq = 0.f;
+                int cnt_gt = 0, n_eq = 0;
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) {
+                    mass_gt += (key[e] > kp) ? pv(e) : 0.f;
+                    cnt_gt += (key[e] > kp) ? 1 : 0;
+                    n_eq += (key[e] == kp) ? 1 : 0;
+                    if (key[e] == kp) p_eq = pv(e);
+                }
+                mass_gt = warp_sum(mass_gt);
+                cnt_gt = (int)__reduce_add_sync(0xFFFFFFFFu, (uint32_t)cnt_gt);
+                n_eq = (int)__reduce_add_sync(0xFFFFFFFFu, (uint32_t)n_eq);
+                p_eq = warp_max(p_eq);
+                // blocks tied at the boundary enter one at a time, lowest index first
+                float accm = mass_gt;
+                int n = 0;
+                while (n < n_eq && accm < target) {
+                    accm += p_eq;
+                    ++n;
+                }
+                const int m_p = cnt_gt + n;
+                const int m = max(m_p, k_min);
+                if (m >= nb) {
+                    all_sel = true;
+                } else if (m == m_p) {
+                    kap = kp;
+                    ntie = n;
+                } else {
+                    // Top-k floor binds: the key of rank m (binary search on counts)
+                    uint32_t lo2 = kmin, hi2 = kp + 1u;  // count(>= lo2) >= m > count(>= hi2)
+                    while (hi2 - lo2 > 1u) {
+                        const uint32_t mid = lo2 + ((hi2 - lo2) >> 1);
+                        uint32_t cc = 0;
+#pragma unroll
+                        for (int e = 0; e < EPL; ++e) cc += (key[e] >= mid) ? 1u : 0u;
+                        if (__reduce_add_sync(0xFFFFFFFFu, cc) >= (uint32_t)m) lo2 = mid;
+                        else hi2 = mid;
+                    }
+                    kap = lo2;
+                    int c_gt = 0;
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) c_gt += (key[e] > kap) ? 1 : 0;
+                    ntie = m - (int)__reduce_add_sync(0xFFFFFFFFu, (uint32_t)c_gt);
+                }
             }
         }
         // ---- compaction in ascending block order (+ diagonal repair)
@@ -373,26 +535,62 @@ __global__ void __launch_bounds__(256) score_select_kernel(Geo g, const float *_
             const uint32_t sm = __ballot_sync(0xFFFFFFFFu, sel);
             if (sel) out[base + __popc(sm & lt_mask)] = j;
             base += __popc(sm);
-            if (probs && valid) probs[row * nb + j] = pv[e] * invz;
+            if (probs && valid) {
+                float pj;
+                if constexpr (kSortedSelect<EPL>) pj = expf(key_float(key[e]) - mx);
+                else pj = srow[j];
+                probs[row * nb + j] = pj * invz;
+            }
         }
         if (lane == 0) kv_cnt[row] = base;
     }
 }
 
+template <int D, int EPL>
+__global__ void __launch_bounds__(256) score_select_kernel(Geo g, const float *__restrict__ qbar,
+                                                           const float *__restrict__ kbarT, float p, int k_min,
+                                                           int32_t *__restrict__ kv_cnt, int32_t *__restrict__ kv_idx,
+                                                           float *__restrict__ probs, uint32_t *__restrict__ status)
+{
+    extern __shared__ __align__(16) float sel_smem[];
+    select_rows<D, EPL>(g, blockIdx.y, blockIdx.x * kSelRows, sel_smem, qbar, kbarT, p, k_min, kv_cnt, kv_idx, probs,
+                        status);
+}
+
 // ---------------------------------------------------------------------------
+template <int D, int NS>
+static cudaError_t launch_pool_t(const Geo &g, int nxs, const void *q, const void *k, float *qbar, float *kbarT,
+                                 cudaStream_t stream)
+{
+    const size_t smem = (size_t)kPoolThreads * NS * 8 * sizeof(float);
+    auto kern = pool_kernel<D, NS>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    const long long blocks = 2ll * g.BH * g.nbt * g.nbh * nxs;
+    kern<<<(unsigned)blocks, kPoolThreads, smem, stream>>>(g, nxs, (const __nv_bfloat16 *)q,
+                                                          (const __nv_bfloat16 *)k, qbar, kbarT);
+    return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_pool_d(const Geo &g, const void *q, const void *k, float *qbar, float *kbarT,
+                                 cudaStream_t stream)
+{
+    const PoolPlan pl = pool_plan(g.nbw, g.bw, D);
+    switch (pl.ns) {
+    case 1: return launch_pool_t<D, 1>(g, pl.nxs, q, k, qbar, kbarT, stream);
+    case 2: return launch_pool_t<D, 2>(g, pl.nxs, q, k, qbar, kbarT, stream);
+    case 3: return launch_pool_t<D, 3>(g, pl.nxs, q, k, qbar, kbarT, stream);
+    case 4: return launch_pool_t<D, 4>(g, pl.nxs, q, k, qbar, kbarT, stream);
+    default: return launch_pool_t<D, 8>(g, pl.nxs, q, k, qbar, kbarT, stream);
+    }
+}
+
 cudaError_t launch_pool(const Geo &g, const void *q, const void *k, float *qbar, float *kbarT,
                         cudaStream_t stream)
 {
-    const long long warps = 2ll * g.BH * g.nb;
-    const int threads = 256;
-    const long long blocks = (warps * 32 + threads - 1) / threads;
-    if (g.D == 128)
-        pool_kernel<128><<<(unsigned)blocks, threads, 0, stream>>>(g, (const __nv_bfloat16 *)q,
-                                                                   (const __nv_bfloat16 *)k, qbar, kbarT);
-    else
-        pool_kernel<64><<<(unsigned)blocks, threads, 0, stream>>>(g, (const __nv_bfloat16 *)q,
-                                                                  (const __nv_bfloat16 *)k, qbar, kbarT);
-    return cudaGetLastError();
+    if (g.D == 128) return launch_pool_d<128>(g, q, k, qbar, kbarT, stream);
+    return launch_pool_d<64>(g, q, k, qbar, kbarT, stream);
 }
 
 template <int D, int EPL>
@@ -400,13 +598,23 @@ static cudaError_t launch_sel_t(const Geo &g, const float *qbar, const float *kb
                                 int32_t *kv_cnt, int32_t *kv_idx, float *probs, uint32_t *status,
                                 cudaStream_t stream)
 {
-    const size_t smem = (size_t)(D * kSelRows + kSelRows * g.nbp) * sizeof(float);
+    const size_t smem = (size_t)(D + sel_slices(g.nbp) * g.nbp) * kSelRows * sizeof(float);
     auto kern = score_select_kernel<D, EPL>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    dim3 grid((unsigned)ceil_div(g.nb, kSelRows), (unsigned)g.BH);
-    kern<<<grid, 256, smem, stream>>>(g, qbar, kbarT, p, k_min, kv_cnt, kv_idx, probs, status);
-    return cudaGetLastError();
+    // programmatic dependent launch: the CTAs may be scheduled while the
+    // pooling kernel drains and wait in-kernel for its results
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)ceil_div(g.nb, kSelRows), (unsigned)g.BH);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, g, qbar, kbarT, p, k_min, kv_cnt, kv_idx, probs, status);
 }
 
 template <int D>

@@ -98,7 +98,9 @@ FVATTN_API int32_t fvattn_default_num_ctas(void);
  * CTAs (0 = fvattn_default_num_ctas()). Returns 0 if the problem is invalid. */
 FVATTN_API size_t fvattn_workspace_size(const fvattn_problem *prob, int32_t num_ctas);
 
-/* Zero the workspace header (status word and counters). Asynchronous. */
+/* Zero the workspace header: the status word and the work counters the
+ * kernels use (the kernels leave the counters at zero when they finish).
+ * Asynchronous. */
 FVATTN_API fvattn_status fvattn_workspace_init(void *ws, size_t ws_bytes, fvattn_stream_t stream);
 
 /*
