@@ -255,6 +255,123 @@ __device__ __forceinline__ uint32_t key_at(const uint32_t (&key)[EPL], int r)
     return __shfl_sync(0xFFFFFFFFu, mine, r / EPL);
 }
 
+// Boundary of the kept set of one row, found over the key space. Block j =
+// lane + 32e of the row has key[e] (0 past the row) and mass pv(e).
+//   MASS:  f(t) = mass(key >= t), goal p*z: the Top-p set;
+//   COUNT: f(t) = count(key >= t), goal m: the m largest keys.
+// On entry f(lo) >= goal > f(hi). Bisection narrows [lo, hi) until it holds
+// at most 32 keys (checked every other step from step kPruneAfter on); those
+// are compacted to one per lane and sorted, and the boundary is read off
+// a prefix scan of their masses (MASS) or their ranks (COUNT). Every key at or
+// above hi is kept. Out: kap, the smallest kept key; ntie, the number of
+// kept blocks whose key equals kap; m_out, the number of kept blocks.
+constexpr int kPruneAfter = 8;
+
+template <int EPL, bool MASS, class PV>
+__device__ __forceinline__ void window_boundary(const uint32_t (&key)[EPL], const PV &pv, float mx, float target,
+                                                int m_goal, uint32_t lo, uint32_t hi, uint32_t *wscr, int lane,
+                                                uint32_t &kap, int &ntie, int &m_out)
+{
+    auto reaches = [&](uint32_t t) {
+        if constexpr (MASS) {
+            float mm = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) mm += (key[e] >= t) ? pv(e) : 0.f;
+            return warp_sum(mm) >= target;
+        } else {
+            uint32_t c = 0;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) c += (key[e] >= t) ? 1u : 0u;
+            return __reduce_add_sync(0xFFFFFFFFu, c) >= (uint32_t)m_goal;
+        }
+    };
+    int steps = 0;
+    while (hi - lo > 1u) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        if (reaches(mid)) lo = mid;
+        else hi = mid;
+        if (++steps >= kPruneAfter && !(steps & 1)) {
+            uint32_t c = 0;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) c += (key[e] >= lo && key[e] < hi) ? 1u : 0u;
+            if (__reduce_add_sync(0xFFFFFFFFu, c) <= 32u) break;
+        }
+    }
+    // blocks with key >= hi are all kept: f(hi) < goal
+    float mass_hi = 0.f;
+    uint32_t cnt_hi = 0;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+        if (key[e] >= hi) {
+            ++cnt_hi;
+            if constexpr (MASS) mass_hi += pv(e);
+        }
+    }
+    cnt_hi = __reduce_add_sync(0xFFFFFFFFu, cnt_hi);
+    if constexpr (MASS) mass_hi = warp_sum(mass_hi);
+    if (hi - lo == 1u) {
+        // one key value left: tied blocks enter one at a time
+        kap = lo;
+        if constexpr (MASS) {
+            float p_eq = 0.f;
+            uint32_t n_eq = 0;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) {
+                if (key[e] == lo) {
+                    ++n_eq;
+                    p_eq = pv(e);
+                }
+            }
+            n_eq = __reduce_add_sync(0xFFFFFFFFu, n_eq);
+            p_eq = warp_max(p_eq);
+            float accm = mass_hi;
+            int n = 0;
+            while (n < (int)n_eq && accm < target) {
+                accm += p_eq;
+                ++n;
+            }
+            ntie = n;
+            m_out = (int)cnt_hi + n;
+        } else {
+            ntie = m_goal - (int)cnt_hi;
+            m_out = m_goal;
+        }
+        return;
+    }
+    // at most 32 keys in [lo, hi): one per lane, sorted descending
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    int nc = 0;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+        const bool in = key[e] >= lo && key[e] < hi;
+        const uint32_t bal = __ballot_sync(0xFFFFFFFFu, in);
+        if (in) wscr[nc + __popc(bal & lt_mask)] = key[e];
+        nc += __popc(bal);
+    }
+    __syncwarp();
+    uint32_t ck[1] = {lane < nc ? wscr[lane] : 0u};
+    __syncwarp();
+    warp_sort_desc<1>(ck, lane);
+    int nk;  // kept candidates: a prefix of the sorted ones
+    if constexpr (MASS) {
+        const float cp = ck[0] ? expf(key_float(ck[0]) - mx) : 0.f;  // the same value as pv of that block
+        float incl = cp;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        float excl = __shfl_up_sync(0xFFFFFFFFu, incl, 1);
+        if (lane == 0) excl = 0.f;
+        nk = __popc(__ballot_sync(0xFFFFFFFFu, ck[0] != 0u && mass_hi + excl < target));
+    } else {
+        nk = m_goal - (int)cnt_hi;
+    }
+    kap = __shfl_sync(0xFFFFFFFFu, ck[0], nk - 1);
+    ntie = nk - __popc(__ballot_sync(0xFFFFFFFFu, ck[0] > kap));
+    m_out = (int)cnt_hi + nk;
+}
+
 // The d range of the score dot products is cut into S slices so that all
 // 256 threads work on small tiles: thread w owns 4 consecutive key blocks x
 // kSelRows rows over one slice (the slice's loads are all in flight at once
@@ -359,6 +476,7 @@ __device__ __forceinline__ void select_rows(const Geo &g, int bh, int i0, float 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t lt_mask = (1u << lane) - 1u;
     const int nb = g.nb;
+    uint32_t *wscr = reinterpret_cast<uint32_t *>(qsT) + warp * 32;  // per-warp scratch; qsT is dead now
     for (int r = warp; r < nrow; r += blockDim.x >> 5) {
         const int i = i0 + r;
         const size_t row = (size_t)bh * nb + i;
@@ -441,7 +559,7 @@ __device__ __forceinline__ void select_rows(const Geo &g, int bh, int i0, float 
                 }
             }
         } else {
-            // Binary search over the key space: the largest key t whose mass
+            // Search over the key space: the largest key t whose mass
             // mass(key >= t) reaches p * z is the Top-p boundary. The masses
             // replace the scores in the row's shared memory.
             uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
@@ -464,59 +582,19 @@ __device__ __forceinline__ void select_rows(const Geo &g, int bh, int i0, float 
             kmax = warp_max_u(kmax);
             if (!all_sel) {
                 const float target = p * z;
-                uint32_t lo = kmin, hi = kmax + 1u;  // mass(>= lo) >= target > mass(>= hi)
-                while (hi - lo > 1u) {
-                    const uint32_t mid = lo + ((hi - lo) >> 1);
-                    float mm = 0.f;
-#pragma unroll
-                    for (int e = 0; e < EPL; ++e) mm += (key[e] >= mid) ? pv(e) : 0.f;
-                    if (warp_sum(mm) >= target) lo = mid;
-                    else hi = mid;
-                }
-                const uint32_t kp = lo;
-                float mass_gt = 0.f, p_eq = 0.f;
-                int cnt_gt = 0, n_eq = 0;
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) {
-                    mass_gt += (key[e] > kp) ? pv(e) : 0.f;
-                    cnt_gt += (key[e] > kp) ? 1 : 0;
-                    n_eq += (key[e] == kp) ? 1 : 0;
-                    if (key[e] == kp) p_eq = pv(e);
-                }
-                mass_gt = warp_sum(mass_gt);
-                cnt_gt = (int)__reduce_add_sync(0xFFFFFFFFu, (uint32_t)cnt_gt);
-                n_eq = (int)__reduce_add_sync(0xFFFFFFFFu, (uint32_t)n_eq);
-                p_eq = warp_max(p_eq);
-                // blocks tied at the boundary enter one at a time, lowest index first
-                float accm = mass_gt;
-                int n = 0;
-                while (n < n_eq && accm < target) {
-                    accm += p_eq;
-                    ++n;
-                }
-                const int m_p = cnt_gt + n;
+                uint32_t kap_p;
+                int ntie_p, m_p;
+                window_boundary<EPL, true>(key, pv, mx, target, 0, kmin, kmax + 1u, wscr, lane, kap_p, ntie_p, m_p);
                 const int m = max(m_p, k_min);
                 if (m >= nb) {
                     all_sel = true;
                 } else if (m == m_p) {
-                    kap = kp;
-                    ntie = n;
+                    kap = kap_p;
+                    ntie = ntie_p;
                 } else {
-                    // Top-k floor binds: the key of rank m (binary search on counts)
-                    uint32_t lo2 = kmin, hi2 = kp + 1u;  // count(>= lo2) >= m > count(>= hi2)
-                    while (hi2 - lo2 > 1u) {
-                        const uint32_t mid = lo2 + ((hi2 - lo2) >> 1);
-                        uint32_t cc = 0;
-#pragma unroll
-                        for (int e = 0; e < EPL; ++e) cc += (key[e] >= mid) ? 1u : 0u;
-                        if (__reduce_add_sync(0xFFFFFFFFu, cc) >= (uint32_t)m) lo2 = mid;
-                        else hi2 = mid;
-                    }
-                    kap = lo2;
-                    int c_gt = 0;
-#pragma unroll
-                    for (int e = 0; e < EPL; ++e) c_gt += (key[e] > kap) ? 1 : 0;
-                    ntie = m - (int)__reduce_add_sync(0xFFFFFFFFu, (uint32_t)c_gt);
+                    // Top-k floor binds: the key of rank m; count(>= kap_p + 1) = m_p - ntie_p < m
+                    int m_c;
+                    window_boundary<EPL, false>(key, pv, mx, 0.f, m, kmin, kap_p + 1u, wscr, lane, kap, ntie, m_c);
                 }
             }
         }

@@ -125,3 +125,60 @@ def test_repeatable():
     assert torch.equal(o1, o2)
     mask = torch.arange(eng.nb, device="cuda")[None, None, None, :] < c1[..., None]
     assert torch.equal(torch.where(mask, i1, 0), torch.where(mask, eng.kv_idx, 0))
+
+
+def _palette_inputs(grid, block, H, D, n_q, n_k, amp, seed):
+    """Every token of a block is the same vector, drawn from a small palette
+    per head, so block means -- and with them block scores -- tie exactly, in
+    fp32 as in fp64 (the grid is a multiple of the block)."""
+    T, Hg, W = grid
+    bt, bh, bw = block
+    nbh, nbw = Hg // bh, W // bw
+    g = torch.Generator().manual_seed(seed)
+    nb = (T // bt) * nbh * nbw
+    pal_q = (torch.randn(H, n_q, D, generator=g) * amp).to(torch.bfloat16)
+    pal_k = (torch.randn(H, n_k, D, generator=g) * amp).to(torch.bfloat16)
+    c_q = torch.randint(n_q, (H, nb), generator=g)
+    c_k = torch.randint(n_k, (H, nb), generator=g)
+    t, y, x = torch.arange(T) // bt, torch.arange(Hg) // bh, torch.arange(W) // bw
+    blk = ((t[:, None, None] * nbh + y[None, :, None]) * nbw + x[None, None, :]).reshape(-1)
+    q = torch.stack([pal_q[h][c_q[h][blk]] for h in range(H)])[None]
+    k = torch.stack([pal_k[h][c_k[h][blk]] for h in range(H)])[None]
+    v = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    return q, k, v
+
+
+@pytest.mark.parametrize("grid,n_k,k_min", [((16, 64, 64), 4, 5), ((16, 64, 64), 40, 24), ((24, 64, 64), 4, 5),
+                                            ((24, 64, 64), 40, 24)])
+def test_exact_score_ties_follow_block_order(grid, n_k, k_min):
+    # Blocks whose scores tie exactly are ranked by block index (lower first),
+    # at the Top-p boundary and at the Top-k floor alike; 256 blocks take the
+    # warp-sort selection, 384 the key-space search
+    import oracle
+    block, H, D, p = (4, 8, 8), 2, 128, 0.6
+    q, k, v = _palette_inputs(grid, block, H, D, 24, n_k, 1.5, seed=37 + n_k)
+    wl = gen.custom("ties", 1, H, D, grid, block, p, k_min, seed=0)
+    eng = _engine(wl)
+    eng.route(q.cuda(), k.cuda())
+    torch.cuda.synchronize()
+    assert eng.status() == 0
+    orc = oracle.get()
+    g = orc.geom(1, H, grid, block, D)
+    qb, kb = orc.pool(g, q), orc.pool(g, k)
+    scale = 1.0 / math.sqrt(D)
+    r = orc.route(g, qb, kb, scale, p, k_min)
+    cmp = fvtest.compare_lists(eng.kv_cnt.cpu().numpy(), eng.kv_idx.cpu().numpy(), r, qb, kb, scale, p, k_min)
+    assert cmp.unexcused == 0, cmp.first_unexcused
+    assert cmp.excused_tie == 0, cmp
+    # the case is meaningful: many rows have an exact tie across their boundary
+    nb = eng.nb
+    s = scale * np.einsum("bhid,bhjd->bhij", qb, kb)
+    order, cnt = r["order"], r["kv_cnt"]
+    tied = 0
+    for h in range(H):
+        for i in range(nb):
+            m = int(cnt[0, h, i])
+            o = order[0, h, i]
+            if 0 < m < nb and s[0, h, i, o[m - 1]] == s[0, h, i, o[min(m, nb - 1)]]:
+                tied += 1
+    assert tied >= nb // 4, tied
