@@ -323,6 +323,7 @@ def run_gpu(args, wl, world, rank, local):
     F = kept_flops(wl, cnt, idx, vs)
     nb = eng.nb
     U = wl.B * wl.H * nb
+    paired = wl.block[0] * wl.block[1] * wl.block[2] == 64  # 64-token blocks run paired query tiles
     dense_F = 4 * wl.D * wl.B * wl.H * wl.N * wl.N
     route_bytes = 2 * wl.B * wl.H * wl.N * wl.D * 2 + 4 * U + 4 * int(cnt.sum())
 
@@ -430,13 +431,14 @@ def run_gpu(args, wl, world, rank, local):
         "density_kept_flops": F / dense_F, "kept_flops_per_step": F, "device_status": status,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": attn_tflops / peak_tf, "traffic": traffic,
-                     "kernel": "attn_kernel<128,128> (fvattn_sparse_attn)",
+                     "kernel": f"attn_kernel<{wl.D},128,{'paired' if paired else 'unpaired'}> (fvattn_sparse_attn)",
                      "peak_source": f"{pk_src} bf16 burst" + ("" if pk_src == "measured" else " (fallback)")},
         "route_roofline": {"bound": "hbm", "achieved": route_bytes / (route_avg * 1e-3) / 1e9,
                            "peak": pk["hbm_gbs"], "unit": "GB/s",
                            "frac": route_bytes / (route_avg * 1e-3) / 1e9 / pk["hbm_gbs"]},
         "clocks": clk,
-        "gpu_launches": 5 * args.steps,
+        # per step: pool + select (route), [pair lists +] two scheduler kernels, attention
+        "gpu_launches": (6 if paired else 5) * args.steps,
         "e2e": e2e,
         "cpu_baseline": cpu,
     }

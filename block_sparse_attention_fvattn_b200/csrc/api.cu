@@ -32,6 +32,8 @@ WsLayout ws_layout(const Geo &g)
     L.unit_cost = take((size_t)g.BH * g.nb * sizeof(int32_t));
     L.head_sorted = take((size_t)g.BH * g.nb * sizeof(int32_t));
     L.head_cost = take((size_t)g.BH * sizeof(int64_t));
+    L.pair_cnt = take(g.paired ? (size_t)g.BH * g.npair * sizeof(int32_t) : 0);
+    L.pair_list = take(g.paired ? (size_t)g.BH * g.npair * g.nb * sizeof(int32_t) : 0);
     L.total = off;
     return L;
 }
@@ -81,6 +83,9 @@ static fvattn_status resolve(const fvattn_problem *p, Geo *g)
         G.nsub = 1;
         G.rows = 64;
     }
+    G.paired = G.rows == 64;
+    G.npair = G.paired ? ceil_div(G.nb, 2) : 0;
+    G.upb = G.paired ? ceil_div(G.nb, 4) : G.nb;
     G.scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / sqrtf((float)G.D);
     G.fd_nbw = make_fastdiv((uint32_t)G.nbw);
     G.fd_hw = make_fastdiv((uint32_t)(G.nbh * G.nbw));
@@ -189,9 +194,16 @@ fvattn_status fvattn_schedule(const fvattn_problem *prob, const int32_t *kv_cnt,
     }
     const WsLayout L = ws_layout(g);
     uint8_t *w = static_cast<uint8_t *>(ws);
+    int32_t *pair_cnt = reinterpret_cast<int32_t *>(w + L.pair_cnt);
+    // paired mode: the unions of the pairs' lists are the attention's work
+    // lists; build them here (the costs need their sizes) for fvattn_sparse_attn
+    if (g.paired && !dense &&
+        launch_pair_lists(g, kv_cnt, kv_idx, pair_cnt, reinterpret_cast<int32_t *>(w + L.pair_list), s) !=
+            cudaSuccess)
+        return FVATTN_ERR_CUDA;
     if (launch_schedule(g, kv_cnt, kv_idx, dense ? 1 : 0, num_ctas, work, cta_range, cta_cost,
                         reinterpret_cast<int32_t *>(w + L.unit_cost), reinterpret_cast<int32_t *>(w + L.head_sorted),
-                        reinterpret_cast<int64_t *>(w + L.head_cost), s) != cudaSuccess)
+                        reinterpret_cast<int64_t *>(w + L.head_cost), pair_cnt, s) != cudaSuccess)
         return FVATTN_ERR_CUDA;
     return FVATTN_OK;
 }
@@ -217,9 +229,17 @@ fvattn_status fvattn_sparse_attn(const fvattn_problem *prob, const void *q, cons
     }
     if (g.BH == 0) return FVATTN_OK;
     uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+    const WsLayout L = ws_layout(g);
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    int32_t *pair_cnt = reinterpret_cast<int32_t *>(w + L.pair_cnt);
+    int32_t *pair_list = reinterpret_cast<int32_t *>(w + L.pair_list);
+    cudaStream_t s = (cudaStream_t)stream;
+    // paired mode without work lists: no fvattn_schedule built the pair lists
+    if (g.paired && !dense && !work && launch_pair_lists(g, kv_cnt, kv_idx, pair_cnt, pair_list, s) != cudaSuccess)
+        return FVATTN_ERR_CUDA;
     int kind = 0;
-    if (launch_attn(g, q, k, v, kv_cnt, kv_idx, work, cta_range, num_ctas, dense ? 1 : 0, out, cta_ns, status,
-                    (cudaStream_t)stream, &kind) != cudaSuccess)
+    if (launch_attn(g, q, k, v, kv_cnt, kv_idx, pair_cnt, pair_list, work, cta_range, num_ctas, dense ? 1 : 0, out,
+                    cta_ns, status, s, &kind) != cudaSuccess)
         return FVATTN_ERR_CUDA;
     return FVATTN_OK;
 }

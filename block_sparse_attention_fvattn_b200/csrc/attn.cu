@@ -7,10 +7,15 @@
 // runs every block through the same code (the guide's VSA_ALL_BLOCKS route).
 //
 // Work unit = one (b, h, query block i). A 256-token block is two 128-row
-// query tiles (its two halves along t), a 64-token block one 64-row tile.
-// Key/value blocks are consumed in sub-tiles of 128 (or 64) tokens, so one
-// 256-token key block is two sub-tiles; a sub-tile that lies wholly outside
-// the grid is skipped, partial ones mask their padded columns.
+// query tiles (its two halves along t), and key/value blocks are consumed in
+// sub-tiles of 128 tokens, so one 256-token key block is two sub-tiles; a
+// sub-tile that lies wholly outside the grid is skipped, partial ones mask
+// their padded columns.
+// 64-token blocks run paired: query blocks (2p, 2p+1) share one 128-row tile
+// (rows 0-63 and 64-127) and walk the union of their two kept lists two key
+// blocks (128 tokens) at a time; each row masks the key blocks its own query
+// block did not keep. A unit is then four query blocks, i.e. two such tiles
+// with separate key/value streams, interleaved tile by tile.
 //
 // Tiles come straight from the raster [B,H,N,D] layout: each tensor is seen
 // by TMA as 5-D (D, W, H, T, B*H) and one sub-tile is one box of
@@ -71,7 +76,7 @@ struct RegSplit {
     static_assert(128 * kLow + 256 * kHigh <= kThreads * kLaunchRegs, "register split exceeds the launch budget");
 };
 
-template <int D, int BKV>
+template <int D, int BKV, bool PAIRED = false>
 struct AttnLayout {
     static constexpr int kDH = D / 64;              // 128-byte column slabs per row
     static constexpr int kQSlab = 128 * 128;        // bytes of one 128-row slab
@@ -80,7 +85,9 @@ struct AttnLayout {
     static constexpr int kK = kQ + 2 * kDH * kQSlab;
     static constexpr int kV = kK + kNK * kDH * kKVSlab;
     static constexpr int kMask = kV + kNV * kDH * kKVSlab;
-    static constexpr int kMaskWords = BKV / 32;
+    // column masks cover one key block of the tile: all BKV columns, or one
+    // 64-token block in paired mode
+    static constexpr int kMaskWords = (PAIRED ? 64 : BKV) / 32;
     // per-axis column masks: entry v-1 of each axis keeps the columns whose
     // coordinate along that axis is < v; blk_w + blk_h + sub_t <= kMaskEntries
     static constexpr int kMaskEntries = 40;
@@ -158,6 +165,61 @@ struct TileCursor {
     }
 };
 
+// Paired mode: unit u = query blocks 4q .. 4q+3 of head bh; tile half h runs
+// pair 2q+h, i.e. query blocks 4q+2h (rows 0-63) and 4q+2h+1 (rows 64-127).
+struct PairUnit {
+    int bh, q;
+    int c0, c1;                  // union size of each half's pair (0: no query block)
+    const int32_t *l0, *l1;      // the unions; nullptr in dense mode (entry e = block e, kept by both)
+    // per-half accessors (selects, so that the struct stays in registers)
+    __device__ __forceinline__ int cnt(int h) const { return h ? c1 : c0; }
+    __device__ __forceinline__ int tiles(int h) const { return (cnt(h) + 1) >> 1; }
+    __device__ __forceinline__ const int32_t *list(int h) const { return h ? l1 : l0; }
+};
+
+__device__ __forceinline__ PairUnit load_pair_unit(const Geo &g, int u, const int32_t *pair_cnt,
+                                                   const int32_t *pair_list, int dense)
+{
+    PairUnit P;
+    P.bh = u / g.upb;
+    P.q = u - P.bh * g.upb;
+    P.c0 = P.c1 = 0;
+    P.l0 = P.l1 = nullptr;
+    for (int h = 0; h < 2; ++h) {
+        const int pp = 2 * P.q + h;
+        int c = 0;
+        const int32_t *lst = nullptr;
+        if (pp < g.npair) {
+            if (dense) {
+                c = g.nb;
+            } else {
+                const size_t pid = (size_t)P.bh * g.npair + pp;
+                c = __ldg(pair_cnt + pid);
+                lst = pair_list + pid * g.nb;
+            }
+        }
+        if (h) {
+            P.c1 = c;
+            P.l1 = lst;
+        } else {
+            P.c0 = c;
+            P.l0 = lst;
+        }
+    }
+    return P;
+}
+
+// Entry e of a union of c entries. Past the end (the second block of an odd
+// last tile) it repeats the last block with no keeper, so that block's
+// columns are masked out for every row.
+__device__ __forceinline__ int pair_entry(const int32_t *lst, int c, int e)
+{
+    const bool past = e >= c;
+    const int ee = past ? c - 1 : e;
+    const int v = lst ? __ldg(lst + ee) : (ee | kPairInA | kPairInB);
+    return past ? (v & kPairBlockMask) : v;
+}
+
 // Rank r of the longest-first order -> unit id. The scheduler deals ranks to
 // C = gridDim.x lists in zigzag rounds (rank r sits at position r / C of list
 // zigzag(r)); without a schedule the rank is the unit id itself.
@@ -213,15 +275,17 @@ __device__ __forceinline__ void exp2_poly_x2(uint64_t a, float &p0, float &p1)
     p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
-template <int D, int BKV>
+template <int D, int BKV, bool PAIRED>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, Geo g, const int32_t *__restrict__ kv_cnt,
-                const int32_t *__restrict__ kv_idx, const int32_t *__restrict__ work,
+                const int32_t *__restrict__ kv_idx, const int32_t *__restrict__ pair_cnt,
+                const int32_t *__restrict__ pair_list, const int32_t *__restrict__ work,
                 const int32_t *__restrict__ cta_range, int dense, __nv_bfloat16 *__restrict__ out,
                 int64_t *__restrict__ cta_ns, uint32_t *__restrict__ status)
 {
-    using L = AttnLayout<D, BKV>;
+    static_assert(!PAIRED || BKV == 128, "paired mode runs 128-token key/value tiles");
+    using L = AttnLayout<D, BKV, PAIRED>;
     extern __shared__ uint8_t attn_smem_raw[];
     const uint32_t raw = smem_u32(attn_smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -277,12 +341,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Units are taken dynamically, longest first, from a counter shared by all
     // CTAs (workspace header word 1); the producer thread takes them and hands
     // them to the other roles through the unit ring.
-    const long long n_units = (long long)g.BH * g.nb;
+    const long long n_units = (long long)g.BH * g.upb;
     uint32_t *unit_cursor = status + 1, *ctas_done = status + 2;
     volatile int32_t *unit_slots = reinterpret_cast<volatile int32_t *>(gbase + L::kUnit);
     UnitFeed feed{bar(L::bUFull), unit_slots, 0};
 
     constexpr uint32_t kTileBytes = (uint32_t)L::kDH * BKV * 128u;
+    constexpr uint32_t kHalfRows = 64u * 128u;  // bytes of 64 rows of a slab (paired mode: second block's offset)
     const uint32_t q_bytes = (uint32_t)L::kDH * (uint32_t)g.rows * 128u;
 
     if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(RegSplit<D, BKV>::kLow));
@@ -307,6 +372,70 @@ __global__ void __launch_bounds__(kThreads, 1)
                 unit_slots[slot] = u;
                 mbar_arrive(bar(L::bUFull + slot));  // release: the id is visible to the waiting roles
                 if (u < 0) break;
+                if constexpr (PAIRED) {
+                    const PairUnit P = load_pair_unit(g, u, pair_cnt, pair_list, dense);
+                    for (int h = 0; h < 2 && ok; ++h) {
+                        if (P.cnt(h) == 0) continue;
+                        if (((q_used >> h) & 1u) &&
+                            !mbar_wait(bar(L::bQEmpty + h), ((q_par >> h) & 1u) ^ 1u, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        const int qa = 2 * (2 * P.q + h);  // rows 0-63: block qa, rows 64-127: block qa+1
+                        const int nq = qa + 1 < g.nb ? 2 : 1;
+                        mbar_arrive_expect_tx(bar(L::bQFull + h), (uint32_t)nq * L::kDH * kHalfRows);
+                        for (int s2 = 0; s2 < nq; ++s2) {
+                            int jt, jy, jx;
+                            block_coords(g, qa + s2, jt, jy, jx);
+                            for (int dh = 0; dh < L::kDH; ++dh)
+                                tma_load_5d(sbase + L::kQ + (h * L::kDH + dh) * L::kQSlab + s2 * kHalfRows, &tm_q,
+                                            bar(L::bQFull + h), dh * 64, jx * g.bw, jy * g.bh, jt * g.bt, P.bh);
+                        }
+                        q_par ^= 1u << h;
+                        q_used |= 1u << h;
+                    }
+                    // key/value tiles, the two halves interleaved: round r is tile r of
+                    // half 0, then tile r of half 1 (each while that half has one)
+                    const int rounds = max(P.tiles(0), P.tiles(1));
+                    for (int r = 0; r < rounds && ok; ++r) {
+                        for (int h = 0; h < 2 && ok; ++h) {
+                            if (r >= P.tiles(h)) continue;
+                            const int jb[2] = {pair_entry(P.list(h), P.cnt(h), 2 * r) & kPairBlockMask,
+                                               pair_entry(P.list(h), P.cnt(h), 2 * r + 1) & kPairBlockMask};
+                            const int ks = kc % kNK;
+                            if (kc >= kNK && !mbar_wait(bar(L::bKEmpty + ks), ((kc / kNK) - 1) & 1, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            mbar_arrive_expect_tx(bar(L::bKFull + ks), kTileBytes);
+                            for (int s2 = 0; s2 < 2; ++s2) {
+                                int jt, jy, jx;
+                                block_coords(g, jb[s2], jt, jy, jx);
+                                for (int dh = 0; dh < L::kDH; ++dh)
+                                    tma_load_5d(sbase + L::kK + (ks * L::kDH + dh) * L::kKVSlab + s2 * kHalfRows,
+                                                &tm_k, bar(L::bKFull + ks), dh * 64, jx * g.bw, jy * g.bh,
+                                                jt * g.bt, P.bh);
+                            }
+                            ++kc;
+                            const int vs = vc % kNV;
+                            if (vc >= kNV && !mbar_wait(bar(L::bVEmpty + vs), ((vc / kNV) - 1) & 1, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            mbar_arrive_expect_tx(bar(L::bVFull + vs), kTileBytes);
+                            for (int s2 = 0; s2 < 2; ++s2) {
+                                int jt, jy, jx;
+                                block_coords(g, jb[s2], jt, jy, jx);
+                                for (int dh = 0; dh < L::kDH; ++dh)
+                                    tma_load_5d(sbase + L::kV + (vs * L::kDH + dh) * L::kKVSlab + s2 * kHalfRows,
+                                                &tm_v, bar(L::bVFull + vs), dh * 64, jx * g.bw, jy * g.bh,
+                                                jt * g.bt, P.bh);
+                            }
+                            ++vc;
+                        }
+                    }
+                    continue;
+                }
                 const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
                 const int x0 = U.ix * g.bw, y0 = U.iy * g.bh, t0 = U.it * g.bt;
                 for (int h = 0; h < U.nh && ok; ++h) {
@@ -376,12 +505,51 @@ __global__ void __launch_bounds__(kThreads, 1)
             int kc = 0, qk_count = 0;
             uint32_t ph_q = 0;
             bool ok = true;
+            // S = Q_h K^T over D in K=16 steps; Q and K slabs are K-major, 128B swizzle
+            auto issue_qk = [&](int h, int ks) {
+                const uint64_t kb = k_desc + (uint64_t)((ks * L::kDH * L::kKVSlab) >> 4);
+                const uint64_t qa = q_desc + (uint64_t)((h * L::kDH * L::kQSlab) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off_a = ((kk >> 2) * L::kQSlab + (kk & 3) * 32) >> 4;
+                    const uint32_t off_b = ((kk >> 2) * L::kKVSlab + (kk & 3) * 32) >> 4;
+                    umma_ss(tmem + L::kTmS, qa + off_a, kb + off_b, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+            };
             while (ok) {
                 int slot;
                 const int u = feed.next(abort_flag, ok, slot);
                 if (!ok) break;
                 mbar_arrive(bar(L::bUEmpty + slot));
                 if (u < 0) break;
+                if constexpr (PAIRED) {
+                    const PairUnit P = load_pair_unit(g, u, pair_cnt, pair_list, dense);
+                    for (int h = 0; h < 2 && ok; ++h) {
+                        if (P.cnt(h) == 0) continue;
+                        ok = mbar_wait(bar(L::bQFull + h), (ph_q >> h) & 1u, abort_flag);
+                        ph_q ^= 1u << h;
+                    }
+                    const int rounds = max(P.tiles(0), P.tiles(1));
+                    for (int r = 0; r < rounds && ok; ++r) {
+                        for (int h = 0; h < 2 && ok; ++h) {
+                            if (r >= P.tiles(h)) continue;
+                            const int ks = kc % kNK;
+                            if (!mbar_wait(bar(L::bKFull + ks), (kc / kNK) & 1, abort_flag)) { ok = false; break; }
+                            if (qk_count > 0 && !mbar_wait(bar(L::bSFree), (qk_count - 1) & 1, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            issue_qk(h, ks);
+                            umma_commit(bar(L::bSFull + h));
+                            ++qk_count;
+                            if (r == P.tiles(h) - 1) umma_commit(bar(L::bQEmpty + h));
+                            umma_commit(bar(L::bKEmpty + ks));
+                            ++kc;
+                        }
+                    }
+                    continue;
+                }
                 const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
                 for (int h = 0; h < U.nh && ok; ++h) {
                     ok = mbar_wait(bar(L::bQFull + h), (ph_q >> h) & 1u, abort_flag);
@@ -390,7 +558,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int k = 0; k < U.nkv && ok; ++k) {
                     const int ks = kc % kNK;
                     if (!mbar_wait(bar(L::bKFull + ks), (kc / kNK) & 1, abort_flag)) { ok = false; break; }
-                    const uint64_t kb = k_desc + (uint64_t)((ks * L::kDH * L::kKVSlab) >> 4);
                     for (int h = 0; h < U.nh; ++h) {
                         // S is shared: overwrite it only once the previous S has been
                         // copied into registers by its softmax warpgroup
@@ -399,14 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             break;
                         }
                         tc_fence_after();
-                        const uint64_t qa = q_desc + (uint64_t)((h * L::kDH * L::kQSlab) >> 4);
-                        // S = Q_h K^T over D in K=16 steps; Q and K slabs are K-major, 128B swizzle
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t off_a = ((kk >> 2) * L::kQSlab + (kk & 3) * 32) >> 4;
-                            const uint32_t off_b = ((kk >> 2) * L::kKVSlab + (kk & 3) * 32) >> 4;
-                            umma_ss(tmem + L::kTmS, qa + off_a, kb + off_b, idesc_qk, kk > 0 ? 1u : 0u);
-                        }
+                        issue_qk(h, ks);
                         umma_commit(bar(L::bSFull + h));
                         ++qk_count;
                         if (k == U.nkv - 1) umma_commit(bar(L::bQEmpty + h));
@@ -428,33 +588,67 @@ __global__ void __launch_bounds__(kThreads, 1)
             int vc = 0;
             uint32_t ph_p = 0, ph_oe = 0, o_pend = 0;
             bool ok = true;
+            // O_h (+)= P_h V over the sub-tile in K=16 steps; P_h from TMEM, V MN-major
+            auto issue_pv = [&](int h, int vs, bool first) {
+                const uint64_t vb = v_desc + (uint64_t)((vs * L::kDH * L::kKVSlab) >> 4);
+                const uint32_t d_tmem = tmem + L::tm_o(h), a_tmem = tmem + L::tm_p(h);
+#pragma unroll
+                for (int kk = 0; kk < BKV / 16; ++kk)
+                    umma_ts(d_tmem, a_tmem + kk * 8, vb + (uint64_t)((kk * 16 * 128) >> 4), idesc_pv,
+                            (!first || kk > 0) ? 1u : 0u);
+            };
+            // before the first product of a unit into O_h: the previous unit's
+            // epilogue must have read O_h
+            auto o_free = [&](int h) {
+                if ((o_pend >> h) & 1u) {
+                    if (!mbar_wait(bar(L::bOEmpty + h), (ph_oe >> h) & 1u, abort_flag)) return false;
+                    ph_oe ^= 1u << h;
+                    o_pend &= ~(1u << h);
+                }
+                return true;
+            };
             while (ok) {
                 int slot;
                 const int u = feed.next(abort_flag, ok, slot);
                 if (!ok) break;
                 mbar_arrive(bar(L::bUEmpty + slot));
                 if (u < 0) break;
+                if constexpr (PAIRED) {
+                    const PairUnit P = load_pair_unit(g, u, pair_cnt, pair_list, dense);
+                    const int rounds = max(P.tiles(0), P.tiles(1));
+                    for (int r = 0; r < rounds && ok; ++r) {
+                        for (int h = 0; h < 2 && ok; ++h) {
+                            if (r >= P.tiles(h)) continue;
+                            const int vs = vc % kNV;
+                            if (!mbar_wait(bar(L::bVFull + vs), (vc / kNV) & 1, abort_flag)) { ok = false; break; }
+                            ok = mbar_wait(bar(L::bPFull + h), (ph_p >> h) & 1u, abort_flag);
+                            ph_p ^= 1u << h;
+                            if (ok && r == 0) ok = o_free(h);
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_pv(h, vs, r == 0);
+                            umma_commit(bar(L::bPFree + h));
+                            if (r == P.tiles(h) - 1) {
+                                umma_commit(bar(L::bOFull + h));
+                                o_pend |= 1u << h;
+                            }
+                            umma_commit(bar(L::bVEmpty + vs));
+                            ++vc;
+                        }
+                    }
+                    continue;
+                }
                 const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
                 for (int k = 0; k < U.nkv && ok; ++k) {
                     const int vs = vc % kNV;
                     if (!mbar_wait(bar(L::bVFull + vs), (vc / kNV) & 1, abort_flag)) { ok = false; break; }
-                    const uint64_t vb = v_desc + (uint64_t)((vs * L::kDH * L::kKVSlab) >> 4);
                     for (int h = 0; h < U.nh; ++h) {
                         ok = mbar_wait(bar(L::bPFull + h), (ph_p >> h) & 1u, abort_flag);
                         ph_p ^= 1u << h;
-                        if (ok && k == 0 && ((o_pend >> h) & 1u)) {  // previous unit's epilogue read O_h
-                            ok = mbar_wait(bar(L::bOEmpty + h), (ph_oe >> h) & 1u, abort_flag);
-                            ph_oe ^= 1u << h;
-                            o_pend &= ~(1u << h);
-                        }
+                        if (ok && k == 0) ok = o_free(h);
                         if (!ok) break;
                         tc_fence_after();
-                        // O_h (+)= P_h V over the sub-tile in K=16 steps; P_h from TMEM, V MN-major
-                        const uint32_t d_tmem = tmem + L::tm_o(h), a_tmem = tmem + L::tm_p(h);
-#pragma unroll
-                        for (int kk = 0; kk < BKV / 16; ++kk)
-                            umma_ts(d_tmem, a_tmem + kk * 8, vb + (uint64_t)((kk * 16 * 128) >> 4), idesc_pv,
-                                    (k > 0 || kk > 0) ? 1u : 0u);
+                        issue_pv(h, vs, k == 0);
                         umma_commit(bar(L::bPFree + h));
                         if (k == U.nkv - 1) {
                             umma_commit(bar(L::bOFull + h));
@@ -480,150 +674,121 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tP = tmem + t_lane + L::tm_p(h);
         const uint32_t tO = tmem + t_lane + L::tm_o(h);
         const float sl2 = g.scale * 1.4426950408889634f;
-        // this thread's query row inside a sub-tile
-        const int r_t = row / (g.bh * g.bw), r_y = (row / g.bw) % g.bh, r_x = row % g.bw;
+        // this thread's query row inside a sub-tile (paired mode: inside its
+        // 64-token query block, which is the first of the pair for rows 0-63)
+        const int r64 = PAIRED ? (row & 63) : row;
+        const int r_t = r64 / (g.bh * g.bw), r_y = (r64 / g.bw) % g.bh, r_x = r64 % g.bw;
         int sf = 0, of = 0, pw = 0;  // S tiles received, O tiles received, P tiles written
         bool ok = true;
-        while (ok) {
-            int slot;
-            const int u = feed.next(abort_flag, ok, slot);
-            if (!ok) break;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(L::bUEmpty + slot));  // every lane has read the id
-            if (u < 0) break;
-            const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
-            if (h >= U.nh) continue;
-            const int qt = U.it * g.bt + h * g.subt + r_t, qy = U.iy * g.bh + r_y, qx = U.ix * g.bw + r_x;
-            const bool row_valid = row < g.rows && qt < g.T && qy < g.Hg && qx < g.W;
-            float m = -INFINITY, l = 0.f;
-            int e = 0, s_sub = 0;
-            int j = U.list ? __ldg(U.list) : 0;
-            for (int k = 0; k < U.nkv; ++k) {
-                // the list entry after this one is loaded now and used next iteration
-                const int j_next = (U.list && e + 1 < U.cnt) ? __ldg(U.list + e + 1) : e + 1;
-                int jt, jy, jx;
-                block_coords(g, j, jt, jy, jx);
-                const int wv = min(g.bw, g.W - jx * g.bw), hv = min(g.bh, g.Hg - jy * g.bh);
-                const int tv = min(g.subt, g.T - (jt * g.bt + s_sub * g.subt));
-                const bool full = (wv == g.bw) && (hv == g.bh) && (tv == g.subt);
-                if (!mbar_wait(bar(L::bSFull + h), sf & 1, abort_flag)) { ok = false; break; }
-                ++sf;
-                tc_fence_after();
-                // all BKV columns in one batch, one wait; the register fences keep
-                // every use of the loaded values after the wait
-                uint32_t r[BKV];
+        float m = -INFINITY, l = 0.f;
+        // One key/value tile of this half: S from TMEM, masks, online softmax,
+        // P into TMEM (after the previous PV of this half), lazy O rescale.
+        auto tile = [&](bool first, auto &&apply_mask) -> bool {
+            if (!mbar_wait(bar(L::bSFull + h), sf & 1, abort_flag)) return false;
+            ++sf;
+            tc_fence_after();
+            // all BKV columns in one batch, one wait; the register fences keep
+            // every use of the loaded values after the wait
+            uint32_t r[BKV];
 #pragma unroll
-                for (int c = 0; c < BKV / 32; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(r + c * 32));
-                tmem_wait_ld();
+            for (int c = 0; c < BKV / 32; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(r + c * 32));
+            tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < BKV / 32; ++c) reg_fence32(r + c * 32);
-                // S is in registers: the next QK may overwrite it
-                tc_fence_before();
-                mbar_arrive(bar(L::bSFree));
-                float x[BKV];
+            for (int c = 0; c < BKV / 32; ++c) reg_fence32(r + c * 32);
+            // S is in registers: the next QK may overwrite it
+            tc_fence_before();
+            mbar_arrive(bar(L::bSFree));
+            float x[BKV];
 #pragma unroll
-                for (int c = 0; c < BKV; ++c) x[c] = __uint_as_float(r[c]);
-                if (!full) {
+            for (int c = 0; c < BKV; ++c) x[c] = __uint_as_float(r[c]);
+            apply_mask(x);
+            // row maximum: 8 independent chains of three-input max, then a tree
+            float m8[8];
 #pragma unroll
-                    for (int w = 0; w < L::kMaskWords; ++w) {
-                        const uint32_t word = mask_w[(wv - 1) * L::kMaskWords + w] &
-                                              mask_h[(hv - 1) * L::kMaskWords + w] &
-                                              mask_t[(tv - 1) * L::kMaskWords + w];
+            for (int q8 = 0; q8 < 8; ++q8) m8[q8] = -INFINITY;
 #pragma unroll
-                        for (int b = 0; b < 32; ++b)
-                            if (!((word >> b) & 1u)) x[w * 32 + b] = -INFINITY;
-                    }
-                }
-                // row maximum: 8 independent chains of three-input max, then a tree
-                float m8[8];
+            for (int c = 0; c < BKV; c += 16)
 #pragma unroll
-                for (int q8 = 0; q8 < 8; ++q8) m8[q8] = -INFINITY;
-#pragma unroll
-                for (int c = 0; c < BKV; c += 16)
-#pragma unroll
-                    for (int q8 = 0; q8 < 8; ++q8) m8[q8] = max3f(m8[q8], x[c + 2 * q8], x[c + 2 * q8 + 1]);
-                const float mx = fmaxf(max3f(m8[0], m8[1], m8[2]), max3f(max3f(m8[3], m8[4], m8[5]), m8[6], m8[7]));
-                const float mt = mx * sl2;
-                float alpha = 1.0f;
-                bool rescale = false;
-                if (k == 0) {
+                for (int q8 = 0; q8 < 8; ++q8) m8[q8] = max3f(m8[q8], x[c + 2 * q8], x[c + 2 * q8 + 1]);
+            const float mx = fmaxf(max3f(m8[0], m8[1], m8[2]), max3f(max3f(m8[3], m8[4], m8[5]), m8[6], m8[7]));
+            const float mt = mx * sl2;
+            float alpha = 1.0f;
+            bool rescale = false;
+            if (first) {
+                m = mt;
+            } else {
+                const bool need = mt > m + kRescaleThreshold;
+                rescale = __any_sync(0xFFFFFFFFu, need);
+                if (need) {
+                    alpha = ex2_approx(m - mt);
                     m = mt;
-                } else {
-                    const bool need = mt > m + kRescaleThreshold;
-                    rescale = __any_sync(0xFFFFFFFFu, need);
-                    if (need) {
-                        alpha = ex2_approx(m - mt);
-                        m = mt;
-                        l *= alpha;
-                    }
-                }
-                // p = 2^(x*scale*log2e - m): packed fp32x2 FMA/ADD, MUFU ex2 (or the
-                // polynomial), packed to bf16 pairs in registers first, so this work
-                // overlaps the PV that still reads the previous P_h
-                const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m, -m);
-                uint64_t s4[4] = {0ull, 0ull, 0ull, 0ull};
-                uint32_t pk[BKV / 2];
-#pragma unroll
-                for (int q2 = 0; q2 < BKV / 2; ++q2) {
-                    const uint64_t a = f2_fma(f2_pack(x[2 * q2], x[2 * q2 + 1]), sl2x2, negm2);
-                    float p0, p1;
-                    if ((q2 & 7) < FV_POLY_PAIRS / 2) {
-                        exp2_poly_x2(a, p0, p1);
-                    } else {
-                        float a0, a1;
-                        f2_unpack(a, a0, a1);
-                        p0 = ex2_approx(a0);
-                        p1 = ex2_approx(a1);
-                    }
-                    s4[q2 & 3] = f2_add(s4[q2 & 3], f2_pack(p0, p1));
-                    pk[q2] = pack_bf16x2(p0, p1);
-                }
-                float sum;
-                {
-                    const uint64_t t = f2_add(f2_add(s4[0], s4[1]), f2_add(s4[2], s4[3]));
-                    float t0, t1;
-                    f2_unpack(t, t0, t1);
-                    sum = t0 + t1;
-                }
-                // P_h and O_h are free once the PV of this half's previous sub-tile is done
-                if (pw > 0 && !mbar_wait(bar(L::bPFree + h), (pw - 1) & 1, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-#pragma unroll
-                for (int c = 0; c < BKV / 32; ++c) tmem_st16(tP + c * 16, pk + c * 16);
-                if (rescale) {
-                    // O_h holds the sum up to the previous sub-tile (its PV is done);
-                    // bring it to the new row maximum
-#pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + c * 32, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int v = 0; v < 32; ++v) o[v] = __float_as_uint(__uint_as_float(o[v]) * alpha);
-                        tmem_st32(tO + c * 32, o);
-                    }
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(bar(L::bPFull + h));
-                ++pw;
-                l += sum;
-                if (g.nsub == 2 && s_sub == 0 && jt * g.bt + g.subt < g.T) {
-                    s_sub = 1;
-                } else {
-                    s_sub = 0;
-                    ++e;
-                    j = j_next;
+                    l *= alpha;
                 }
             }
-            if (!ok) break;
-            // epilogue: O / l -> bf16, raster order, valid rows only
-            if (!mbar_wait(bar(L::bOFull + h), of & 1, abort_flag)) { ok = false; break; }
+            // p = 2^(x*scale*log2e - m): packed fp32x2 FMA/ADD, MUFU ex2 (or the
+            // polynomial), packed to bf16 pairs in registers first, so this work
+            // overlaps the PV that still reads the previous P_h
+            // paired mode: a row whose own query block kept no block of the
+            // tiles so far has m = -inf; its p are 0 (not inf - inf)
+            const float m_use = (PAIRED && m == -INFINITY) ? 0.f : m;
+            const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_use, -m_use);
+            uint64_t s4[4] = {0ull, 0ull, 0ull, 0ull};
+            uint32_t pk[BKV / 2];
+#pragma unroll
+            for (int q2 = 0; q2 < BKV / 2; ++q2) {
+                const uint64_t a = f2_fma(f2_pack(x[2 * q2], x[2 * q2 + 1]), sl2x2, negm2);
+                float p0, p1;
+                if ((q2 & 7) < FV_POLY_PAIRS / 2) {
+                    exp2_poly_x2(a, p0, p1);
+                } else {
+                    float a0, a1;
+                    f2_unpack(a, a0, a1);
+                    p0 = ex2_approx(a0);
+                    p1 = ex2_approx(a1);
+                }
+                s4[q2 & 3] = f2_add(s4[q2 & 3], f2_pack(p0, p1));
+                pk[q2] = pack_bf16x2(p0, p1);
+            }
+            float sum;
+            {
+                const uint64_t t = f2_add(f2_add(s4[0], s4[1]), f2_add(s4[2], s4[3]));
+                float t0, t1;
+                f2_unpack(t, t0, t1);
+                sum = t0 + t1;
+            }
+            // P_h and O_h are free once the PV of this half's previous sub-tile is done
+            if (pw > 0 && !mbar_wait(bar(L::bPFree + h), (pw - 1) & 1, abort_flag)) return false;
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < BKV / 32; ++c) tmem_st16(tP + c * 16, pk + c * 16);
+            if (rescale) {
+                // O_h holds the sum up to the previous sub-tile (its PV is done);
+                // bring it to the new row maximum
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + c * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int v = 0; v < 32; ++v) o[v] = __float_as_uint(__uint_as_float(o[v]) * alpha);
+                    tmem_st32(tO + c * 32, o);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(L::bPFull + h));
+            ++pw;
+            l += sum;
+            return true;
+        };
+        // epilogue: O / l -> bf16, raster order, valid rows only
+        auto epilogue = [&](int ubh, int qt, int qy, int qx, bool row_valid) -> bool {
+            if (!mbar_wait(bar(L::bOFull + h), of & 1, abort_flag)) return false;
             ++of;
             tc_fence_after();
             const float inv = 1.0f / l;
             __nv_bfloat16 *orow =
-                out + ((size_t)U.bh * g.N + ((size_t)qt * g.Hg + qy) * g.W + qx) * (size_t)D;
+                out + ((size_t)ubh * g.N + ((size_t)qt * g.Hg + qy) * g.W + qx) * (size_t)D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
@@ -644,6 +809,113 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_before();
             mbar_arrive(bar(L::bOEmpty + h));
+            return true;
+        };
+        while (ok) {
+            int slot;
+            const int u = feed.next(abort_flag, ok, slot);
+            if (!ok) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(L::bUEmpty + slot));  // every lane has read the id
+            if (u < 0) break;
+            if constexpr (PAIRED) {
+                const PairUnit P = load_pair_unit(g, u, pair_cnt, pair_list, dense);
+                const int c_h = P.cnt(h), n_h = P.tiles(h);
+                const int32_t *lst = P.list(h);
+                if (n_h == 0) continue;
+                const int hb = row >> 6;                   // 0: first query block of the pair, 1: second
+                const int qi = 2 * (2 * P.q + h) + hb;     // this row's query block
+                const int keeper = hb ? kPairInB : kPairInA;
+                int it, iy, ix;
+                block_coords(g, qi, it, iy, ix);
+                const int qt = it * g.bt + r_t, qy = iy * g.bh + r_y, qx = ix * g.bw + r_x;
+                const bool row_valid = qi < g.nb && qt < g.T && qy < g.Hg && qx < g.W;
+                m = -INFINITY;
+                l = 0.f;
+                int ent0 = pair_entry(lst, c_h, 0), ent1 = pair_entry(lst, c_h, 1);
+                for (int r = 0; r < n_h; ++r) {
+                    // the next tile's entries are loaded now and used next iteration
+                    const int nxt0 = pair_entry(lst, c_h, 2 * r + 2), nxt1 = pair_entry(lst, c_h, 2 * r + 3);
+                    // column word w covers key block ent(w/2): all masked unless this
+                    // row's query block kept it, then its padding masked
+                    uint32_t mw[4];
+                    bool all = true;
+#pragma unroll
+                    for (int s2 = 0; s2 < 2; ++s2) {
+                        const int ent = s2 ? ent1 : ent0;
+                        int jt, jy, jx;
+                        block_coords(g, ent & kPairBlockMask, jt, jy, jx);
+                        const int wv = min(g.bw, g.W - jx * g.bw), hv = min(g.bh, g.Hg - jy * g.bh);
+                        const int tv = min(g.bt, g.T - jt * g.bt);
+                        const bool keep = (ent & keeper) != 0;
+                        const bool full = wv == g.bw && hv == g.bh && tv == g.bt;
+#pragma unroll
+                        for (int w = 0; w < L::kMaskWords; ++w) {
+                            const uint32_t word = !keep ? 0u
+                                                  : full ? 0xFFFFFFFFu
+                                                         : (mask_w[(wv - 1) * L::kMaskWords + w] &
+                                                            mask_h[(hv - 1) * L::kMaskWords + w] &
+                                                            mask_t[(tv - 1) * L::kMaskWords + w]);
+                            mw[s2 * L::kMaskWords + w] = word;
+                            all = all && word == 0xFFFFFFFFu;
+                        }
+                    }
+                    auto mask = [&](float(&x)[BKV]) {
+                        if (all) return;
+#pragma unroll
+                        for (int w = 0; w < 4; ++w)
+#pragma unroll
+                            for (int b = 0; b < 32; ++b)
+                                if (!((mw[w] >> b) & 1u)) x[w * 32 + b] = -INFINITY;
+                    };
+                    if (!tile(r == 0, mask)) { ok = false; break; }
+                    ent0 = nxt0;
+                    ent1 = nxt1;
+                }
+                if (!ok) break;
+                if (!epilogue(P.bh, qt, qy, qx, row_valid)) { ok = false; break; }
+                continue;
+            }
+            const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
+            if (h >= U.nh) continue;
+            const int qt = U.it * g.bt + h * g.subt + r_t, qy = U.iy * g.bh + r_y, qx = U.ix * g.bw + r_x;
+            const bool row_valid = row < g.rows && qt < g.T && qy < g.Hg && qx < g.W;
+            m = -INFINITY;
+            l = 0.f;
+            int e = 0, s_sub = 0;
+            int j = U.list ? __ldg(U.list) : 0;
+            for (int k = 0; k < U.nkv; ++k) {
+                // the list entry after this one is loaded now and used next iteration
+                const int j_next = (U.list && e + 1 < U.cnt) ? __ldg(U.list + e + 1) : e + 1;
+                int jt, jy, jx;
+                block_coords(g, j, jt, jy, jx);
+                const int wv = min(g.bw, g.W - jx * g.bw), hv = min(g.bh, g.Hg - jy * g.bh);
+                const int tv = min(g.subt, g.T - (jt * g.bt + s_sub * g.subt));
+                const bool full = (wv == g.bw) && (hv == g.bh) && (tv == g.subt);
+                auto mask = [&](float(&x)[BKV]) {
+                    if (!full) {
+    #pragma unroll
+                        for (int w = 0; w < L::kMaskWords; ++w) {
+                            const uint32_t word = mask_w[(wv - 1) * L::kMaskWords + w] &
+                                                  mask_h[(hv - 1) * L::kMaskWords + w] &
+                                                  mask_t[(tv - 1) * L::kMaskWords + w];
+    #pragma unroll
+                            for (int b = 0; b < 32; ++b)
+                                if (!((word >> b) & 1u)) x[w * 32 + b] = -INFINITY;
+                        }
+                    }
+                };
+                if (!tile(k == 0, mask)) { ok = false; break; }
+                if (g.nsub == 2 && s_sub == 0 && jt * g.bt + g.subt < g.T) {
+                    s_sub = 1;
+                } else {
+                    s_sub = 0;
+                    ++e;
+                    j = j_next;
+                }
+            }
+            if (!ok) break;
+            if (!epilogue(U.bh, qt, qy, qx, row_valid)) { ok = false; break; }
         }
     }
 
@@ -700,14 +972,14 @@ static bool make_map(CUtensorMap *map, const Geo &g, const void *ptr)
     return r == CUDA_SUCCESS;
 }
 
-template <int D, int BKV>
+template <int D, int BKV, bool PAIRED>
 static cudaError_t launch_attn_t(const Geo &g, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
-                                 const int32_t *kv_cnt, const int32_t *kv_idx, const int32_t *work,
-                                 const int32_t *cta_range, int grid, int dense, void *out, int64_t *cta_ns,
-                                 uint32_t *status, cudaStream_t stream)
+                                 const int32_t *kv_cnt, const int32_t *kv_idx, const int32_t *pair_cnt,
+                                 const int32_t *pair_list, const int32_t *work, const int32_t *cta_range, int grid,
+                                 int dense, void *out, int64_t *cta_ns, uint32_t *status, cudaStream_t stream)
 {
-    using L = AttnLayout<D, BKV>;
-    auto kern = attn_kernel<D, BKV>;
+    using L = AttnLayout<D, BKV, PAIRED>;
+    auto kern = attn_kernel<D, BKV, PAIRED>;
     cudaFuncAttributes fa;
     cudaError_t err = cudaFuncGetAttributes(&fa, kern);
     if (err != cudaSuccess) return err;
@@ -717,15 +989,15 @@ static cudaError_t launch_attn_t(const Geo &g, const CUtensorMap &mq, const CUte
         return cudaErrorInvalidConfiguration;
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (err != cudaSuccess) return err;
-    kern<<<grid, kThreads, L::kAlloc, stream>>>(mq, mk, mv, g, kv_cnt, kv_idx, work, cta_range, dense,
-                                                (__nv_bfloat16 *)out, cta_ns, status);
+    kern<<<grid, kThreads, L::kAlloc, stream>>>(mq, mk, mv, g, kv_cnt, kv_idx, pair_cnt, pair_list, work, cta_range,
+                                                dense, (__nv_bfloat16 *)out, cta_ns, status);
     return cudaGetLastError();
 }
 
 cudaError_t launch_attn(const Geo &g, const void *q, const void *k, const void *v, const int32_t *kv_cnt,
-                        const int32_t *kv_idx, const int32_t *work, const int32_t *cta_range, int num_ctas,
-                        int dense, void *out, int64_t *cta_ns, uint32_t *status, cudaStream_t stream,
-                        int *launch_error_kind)
+                        const int32_t *kv_idx, const int32_t *pair_cnt, const int32_t *pair_list,
+                        const int32_t *work, const int32_t *cta_range, int num_ctas, int dense, void *out,
+                        int64_t *cta_ns, uint32_t *status, cudaStream_t stream, int *launch_error_kind)
 {
     *launch_error_kind = 0;
     CUtensorMap mq, mk, mv;
@@ -735,21 +1007,21 @@ cudaError_t launch_attn(const Geo &g, const void *q, const void *k, const void *
     }
     int grid = num_ctas;
     if (!work) {
-        const long long U = (long long)g.BH * g.nb;
+        const long long U = (long long)g.BH * g.upb;
         if (U < grid) grid = (int)U;
     }
-    if (g.rows == 128) {
+    if (g.paired) {
         if (g.D == 128)
-            return launch_attn_t<128, 128>(g, mq, mk, mv, kv_cnt, kv_idx, work, cta_range, grid, dense, out, cta_ns,
-                                           status, stream);
-        return launch_attn_t<64, 128>(g, mq, mk, mv, kv_cnt, kv_idx, work, cta_range, grid, dense, out, cta_ns,
-                                      status, stream);
+            return launch_attn_t<128, 128, true>(g, mq, mk, mv, kv_cnt, kv_idx, pair_cnt, pair_list, work, cta_range,
+                                                 grid, dense, out, cta_ns, status, stream);
+        return launch_attn_t<64, 128, true>(g, mq, mk, mv, kv_cnt, kv_idx, pair_cnt, pair_list, work, cta_range,
+                                            grid, dense, out, cta_ns, status, stream);
     }
     if (g.D == 128)
-        return launch_attn_t<128, 64>(g, mq, mk, mv, kv_cnt, kv_idx, work, cta_range, grid, dense, out, cta_ns,
-                                      status, stream);
-    return launch_attn_t<64, 64>(g, mq, mk, mv, kv_cnt, kv_idx, work, cta_range, grid, dense, out, cta_ns, status,
-                                 stream);
+        return launch_attn_t<128, 128, false>(g, mq, mk, mv, kv_cnt, kv_idx, pair_cnt, pair_list, work, cta_range,
+                                              grid, dense, out, cta_ns, status, stream);
+    return launch_attn_t<64, 128, false>(g, mq, mk, mv, kv_cnt, kv_idx, pair_cnt, pair_list, work, cta_range, grid,
+                                         dense, out, cta_ns, status, stream);
 }
 
 }  // namespace fvattn

@@ -45,6 +45,9 @@ struct Geo {
     int subt;              // frames per 128-/64-row sub-tile (bt/2 for 256-token blocks, bt for 64)
     int nsub;              // sub-tiles per block along t (2 or 1)
     int rows;              // rows per sub-tile (128 or 64)
+    int paired;            // 64-token blocks: two query blocks share one 128-row tile
+    int npair;             // pairs of query blocks (2p, 2p+1) per head: ceil(nb/2) when paired
+    int upb;               // attention work units per (b, h): nb, or ceil(nb/4) when paired
     float scale;           // softmax scale
     FastDiv fd_nbw;        // divide by nbw
     FastDiv fd_hw;         // divide by nbh * nbw

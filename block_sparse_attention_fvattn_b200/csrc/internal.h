@@ -15,6 +15,8 @@ struct WsLayout {
     size_t unit_cost;    // int32 [BH*nb]      scheduler: cost per unit
     size_t head_sorted;  // int32 [BH*nb]      scheduler: units of each head by cost
     size_t head_cost;    // int64 [BH]         scheduler: total cost per head
+    size_t pair_cnt;     // int32 [BH*npair]   paired mode: union size of each pair of query blocks
+    size_t pair_list;    // int32 [BH*npair*nb] paired mode: the union, ascending, with membership flags
     size_t total;
 };
 WsLayout ws_layout(const Geo &g);
@@ -31,10 +33,16 @@ cudaError_t launch_score_select(const Geo &g, const float *qbar, const float *kb
                                 cudaStream_t stream);
 cudaError_t launch_schedule(const Geo &g, const int32_t *kv_cnt, const int32_t *kv_idx, int dense, int num_ctas,
                             int32_t *work, int32_t *cta_range, int64_t *cta_cost, int32_t *unit_cost,
-                            int32_t *head_sorted, int64_t *head_cost, cudaStream_t stream);
+                            int32_t *head_sorted, int64_t *head_cost, const int32_t *pair_cnt,
+                            cudaStream_t stream);
+// Paired mode (64-token blocks): entry = block | kPairInA (kept by the first
+// query block of the pair) | kPairInB (kept by the second).
+constexpr int32_t kPairInA = 1 << 16, kPairInB = 1 << 17, kPairBlockMask = 0xFFFF;
+cudaError_t launch_pair_lists(const Geo &g, const int32_t *kv_cnt, const int32_t *kv_idx, int32_t *pair_cnt,
+                              int32_t *pair_list, cudaStream_t stream);
 cudaError_t launch_attn(const Geo &g, const void *q, const void *k, const void *v, const int32_t *kv_cnt,
-                        const int32_t *kv_idx, const int32_t *work, const int32_t *cta_range, int num_ctas,
-                        int dense, void *out, int64_t *cta_ns, uint32_t *status, cudaStream_t stream,
-                        int *launch_error_kind);
+                        const int32_t *kv_idx, const int32_t *pair_cnt, const int32_t *pair_list,
+                        const int32_t *work, const int32_t *cta_range, int num_ctas, int dense, void *out,
+                        int64_t *cta_ns, uint32_t *status, cudaStream_t stream, int *launch_error_kind);
 
 }  // namespace fvattn

@@ -161,7 +161,16 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geo g, int nxs, cons
 
 // ---------------------------------------------------------------------------
 // K2
-constexpr int kSelRows = 8;  // query blocks per CTA (rows of the score tile), one per warp
+// Query blocks per CTA (rows of the score tile). Each CTA reads its head's
+// whole pooled-key matrix once, so rows longer than 1024 blocks take 16 rows
+// per CTA (two per warp) to halve that traffic; shorter rows take 8 (one per
+// warp) to keep more CTAs in flight.
+template <int EPL>
+constexpr int kSelRowsFor = EPL >= 32 ? 16 : 8;
+// CTAs per SM the register budget is sized for (the score tile and the row's
+// keys live in registers).
+template <int EPL>
+constexpr int kSelMinBlocksFor = EPL >= 32 ? 2 : 3;
 // Rows of up to 256 blocks select by a warp sort of their keys; longer rows by
 // a binary search over the key space (fewer passes over the row's elements).
 template <int EPL>
@@ -267,6 +276,17 @@ __device__ __forceinline__ uint32_t key_at(const uint32_t (&key)[EPL], int r)
 // kept blocks whose key equals kap; m_out, the number of kept blocks.
 constexpr int kPruneAfter = 8;
 
+// mass(key >= t) of one row: four interleaved partial sums per lane (short
+// dependency chains), combined in a fixed order, then across the warp.
+template <int EPL, class PV>
+__device__ __forceinline__ float mass_at_least(const uint32_t (&key)[EPL], const PV &pv, uint32_t t)
+{
+    float m[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) m[e & 3] += (key[e] >= t) ? pv(e) : 0.f;
+    return warp_sum((m[0] + m[1]) + (m[2] + m[3]));
+}
+
 template <int EPL, bool MASS, class PV>
 __device__ __forceinline__ void window_boundary(const uint32_t (&key)[EPL], const PV &pv, float mx, float target,
                                                 int m_goal, uint32_t lo, uint32_t hi, uint32_t *wscr, int lane,
@@ -274,10 +294,7 @@ __device__ __forceinline__ void window_boundary(const uint32_t (&key)[EPL], cons
 {
     auto reaches = [&](uint32_t t) {
         if constexpr (MASS) {
-            float mm = 0.f;
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) mm += (key[e] >= t) ? pv(e) : 0.f;
-            return warp_sum(mm) >= target;
+            return mass_at_least<EPL>(key, pv, t) >= target;
         } else {
             uint32_t c = 0;
 #pragma unroll
@@ -297,18 +314,14 @@ __device__ __forceinline__ void window_boundary(const uint32_t (&key)[EPL], cons
             if (__reduce_add_sync(0xFFFFFFFFu, c) <= 32u) break;
         }
     }
-    // blocks with key >= hi are all kept: f(hi) < goal
+    // blocks with key >= hi are all kept: f(hi) < goal (mass_hi is the value
+    // the search compared when it set hi, bit for bit)
     float mass_hi = 0.f;
     uint32_t cnt_hi = 0;
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-        if (key[e] >= hi) {
-            ++cnt_hi;
-            if constexpr (MASS) mass_hi += pv(e);
-        }
-    }
+    for (int e = 0; e < EPL; ++e) cnt_hi += (key[e] >= hi) ? 1u : 0u;
     cnt_hi = __reduce_add_sync(0xFFFFFFFFu, cnt_hi);
-    if constexpr (MASS) mass_hi = warp_sum(mass_hi);
+    if constexpr (MASS) mass_hi = mass_at_least<EPL>(key, pv, hi);
     if (hi - lo == 1u) {
         // one key value left: tied blocks enter one at a time
         kap = lo;
@@ -374,63 +387,69 @@ __device__ __forceinline__ void window_boundary(const uint32_t (&key)[EPL], cons
 
 // The d range of the score dot products is cut into S slices so that all
 // 256 threads work on small tiles: thread w owns 4 consecutive key blocks x
-// kSelRows rows over one slice (the slice's loads are all in flight at once
-// when it is short). Per element the slice sums are fp32 fmas in ascending d,
-// and the slices are then added in ascending order.
+// ROWS rows over one slice (the slice's loads are all in flight at once when
+// it is short), accumulated as row pairs with packed fp32x2 fmas. Per element
+// the slice sums are fp32 fmas in ascending d, and the slices are then added
+// in ascending order.
 __host__ __device__ constexpr int sel_slices(int nbp)
 {
     return (nbp >> 2) >= 256 ? 1 : (nbp >> 2) >= 128 ? 2 : (nbp >> 2) >= 64 ? 4 : 8;
 }
 
-template <int D, int S>
+template <int D, int S, int ROWS>
 __device__ __forceinline__ void score_tile(const float *kb, const float *qsT, float *sc, int nbp, float scale)
 {
     constexpr int DS = D / S;
     constexpr int kUnroll = DS <= 16 ? DS : 8;
+    constexpr int RP = ROWS / 2;  // row pairs: one packed fp32x2 accumulator per pair and column
     const int NQ = nbp >> 2;
     for (int w = threadIdx.x; w < NQ * S; w += blockDim.x) {
         const int sl = S == 1 ? 0 : w / NQ;
         const int c0 = (w - sl * NQ) * 4;
-        uint64_t acc[kSelRows][2];
+        uint64_t acc[RP][4];
 #pragma unroll
-        for (int r = 0; r < kSelRows; ++r) acc[r][0] = acc[r][1] = 0ull;
+        for (int r = 0; r < RP; ++r)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[r][c] = 0ull;
         const float *kp = kb + (size_t)(sl * DS) * nbp + c0;
-        const float *qp = qsT + sl * DS * kSelRows;
+        const float *qp = qsT + sl * DS * ROWS;
 #pragma unroll kUnroll
         for (int d = 0; d < DS; ++d) {
             const float4 kv = __ldg(reinterpret_cast<const float4 *>(kp + (size_t)d * nbp));
-            const uint64_t k01 = f2_pack(kv.x, kv.y), k23 = f2_pack(kv.z, kv.w);
-            const float4 *qv = reinterpret_cast<const float4 *>(qp + d * kSelRows);
+            const uint64_t k2[4] = {f2_pack(kv.x, kv.x), f2_pack(kv.y, kv.y), f2_pack(kv.z, kv.z),
+                                    f2_pack(kv.w, kv.w)};
+            const float4 *qv = reinterpret_cast<const float4 *>(qp + d * ROWS);
 #pragma unroll
-            for (int r4 = 0; r4 < kSelRows / 4; ++r4) {
+            for (int r4 = 0; r4 < ROWS / 4; ++r4) {
                 const float4 qq = qv[r4];
-                const float qr[4] = {qq.x, qq.y, qq.z, qq.w};
+                const uint64_t q01 = f2_pack(qq.x, qq.y), q23 = f2_pack(qq.z, qq.w);
 #pragma unroll
-                for (int rr = 0; rr < 4; ++rr) {
-                    const uint64_t q2 = f2_pack(qr[rr], qr[rr]);
-                    acc[r4 * 4 + rr][0] = f2_fma(q2, k01, acc[r4 * 4 + rr][0]);
-                    acc[r4 * 4 + rr][1] = f2_fma(q2, k23, acc[r4 * 4 + rr][1]);
+                for (int c = 0; c < 4; ++c) {
+                    acc[2 * r4][c] = f2_fma(q01, k2[c], acc[2 * r4][c]);
+                    acc[2 * r4 + 1][c] = f2_fma(q23, k2[c], acc[2 * r4 + 1][c]);
                 }
             }
         }
-        float *dst = sc + (size_t)sl * kSelRows * nbp;
+        float *dst = sc + (size_t)sl * ROWS * nbp;
         const float f = S == 1 ? scale : 1.0f;
 #pragma unroll
-        for (int r = 0; r < kSelRows; ++r) {
-            float a0, a1, a2, a3;
-            f2_unpack(acc[r][0], a0, a1);
-            f2_unpack(acc[r][1], a2, a3);
-            *reinterpret_cast<float4 *>(dst + r * nbp + c0) = make_float4(f * a0, f * a1, f * a2, f * a3);
+        for (int r = 0; r < RP; ++r) {
+            float lo[4], hi[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) f2_unpack(acc[r][c], lo[c], hi[c]);
+            *reinterpret_cast<float4 *>(dst + (2 * r) * nbp + c0) = make_float4(f * lo[0], f * lo[1], f * lo[2], f * lo[3]);
+            *reinterpret_cast<float4 *>(dst + (2 * r + 1) * nbp + c0) =
+                make_float4(f * hi[0], f * hi[1], f * hi[2], f * hi[3]);
         }
     }
     if (S > 1) {
         __syncthreads();
-        const int n4 = kSelRows * nbp / 4;
+        const int n4 = ROWS * nbp / 4;
         for (int x = threadIdx.x; x < n4; x += blockDim.x) {
             float4 t = reinterpret_cast<const float4 *>(sc)[x];
 #pragma unroll
             for (int sl = 1; sl < S; ++sl) {
-                const float4 u = reinterpret_cast<const float4 *>(sc + (size_t)sl * kSelRows * nbp)[x];
+                const float4 u = reinterpret_cast<const float4 *>(sc + (size_t)sl * ROWS * nbp)[x];
                 t.x += u.x;
                 t.y += u.y;
                 t.z += u.z;
@@ -441,35 +460,36 @@ __device__ __forceinline__ void score_tile(const float *kb, const float *qsT, fl
     }
 }
 
-// The CTA (8 warps) routes query blocks i0 .. i0+7 of head bh: scores into
-// shared memory, then one warp per row selects and compacts. Shared memory:
-// (D + sel_slices(nbp) * nbp) * kSelRows floats.
+// The CTA (8 warps) routes query blocks i0 .. i0+ROWS-1 of head bh: scores
+// into shared memory, then each warp selects and compacts whole rows. Shared
+// memory: (D + sel_slices(nbp) * nbp) * ROWS floats.
 template <int D, int EPL>
 __device__ __forceinline__ void select_rows(const Geo &g, int bh, int i0, float *sel_smem,
                                             const float *qbar, const float *kbarT, float p,
                                             int k_min, int32_t *__restrict__ kv_cnt, int32_t *__restrict__ kv_idx,
                                             float *__restrict__ probs, uint32_t *__restrict__ status)
 {
-    float *qsT = sel_smem;                 // [D][kSelRows]
-    float *sc = sel_smem + D * kSelRows;   // [S][kSelRows][nbp]; slice 0 ends up holding the scores
-    const int nrow = min(kSelRows, g.nb - i0);
+    constexpr int ROWS = kSelRowsFor<EPL>;
+    float *qsT = sel_smem;             // [D][ROWS]
+    float *sc = sel_smem + D * ROWS;   // [S][ROWS][nbp]; slice 0 ends up holding the scores
+    const int nrow = min(ROWS, g.nb - i0);
     const int nbp = g.nbp;
 
     // launched as a programmatic dependent of the pooling kernel: wait for it
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    for (int idx = threadIdx.x; idx < kSelRows * D; idx += blockDim.x) {
+    for (int idx = threadIdx.x; idx < ROWS * D; idx += blockDim.x) {
         const int r = idx / D, d = idx - r * D;
-        qsT[d * kSelRows + r] = (r < nrow) ? qbar[((size_t)bh * g.nb + i0 + r) * D + d] : 0.f;
+        qsT[d * ROWS + r] = (r < nrow) ? qbar[((size_t)bh * g.nb + i0 + r) * D + d] : 0.f;
     }
     __syncthreads();
 
     // ---- block scores
     const float *kb = kbarT + (size_t)bh * D * nbp;
     const int S = sel_slices(nbp);
-    if (S == 8) score_tile<D, 8>(kb, qsT, sc, nbp, g.scale);
-    else if (S == 4) score_tile<D, 4>(kb, qsT, sc, nbp, g.scale);
-    else if (S == 2) score_tile<D, 2>(kb, qsT, sc, nbp, g.scale);
-    else score_tile<D, 1>(kb, qsT, sc, nbp, g.scale);
+    if (S == 8) score_tile<D, 8, ROWS>(kb, qsT, sc, nbp, g.scale);
+    else if (S == 4) score_tile<D, 4, ROWS>(kb, qsT, sc, nbp, g.scale);
+    else if (S == 2) score_tile<D, 2, ROWS>(kb, qsT, sc, nbp, g.scale);
+    else score_tile<D, 1, ROWS>(kb, qsT, sc, nbp, g.scale);
     __syncthreads();
 
     // ---- selection: one warp per row
@@ -563,7 +583,7 @@ __device__ __forceinline__ void select_rows(const Geo &g, int bh, int i0, float 
             // mass(key >= t) reaches p * z is the Top-p boundary. The masses
             // replace the scores in the row's shared memory.
             uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-            float zl = 0.f;
+            float zl[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int e = 0; e < EPL; ++e) {
                 const int j = lane + 32 * e;
@@ -572,12 +592,12 @@ __device__ __forceinline__ void select_rows(const Geo &g, int bh, int i0, float 
                     srow[j] = pj;
                     kmin = min(kmin, key[e]);
                     kmax = max(kmax, key[e]);
-                    zl += pj;
+                    zl[e & 3] += pj;
                 }
             }
             const float *pvr = srow;  // pv of block j at pvr[j]; read only where key[e] != 0
             auto pv = [&](int e) { return key[e] ? pvr[lane + 32 * e] : 0.f; };
-            z = warp_sum(zl);
+            z = warp_sum((zl[0] + zl[1]) + (zl[2] + zl[3]));
             kmin = warp_min_u(kmin);
             kmax = warp_max_u(kmax);
             if (!all_sel) {
@@ -625,13 +645,13 @@ __device__ __forceinline__ void select_rows(const Geo &g, int bh, int i0, float 
 }
 
 template <int D, int EPL>
-__global__ void __launch_bounds__(256) score_select_kernel(Geo g, const float *__restrict__ qbar,
+__global__ void __launch_bounds__(256, kSelMinBlocksFor<EPL>) score_select_kernel(Geo g, const float *__restrict__ qbar,
                                                            const float *__restrict__ kbarT, float p, int k_min,
                                                            int32_t *__restrict__ kv_cnt, int32_t *__restrict__ kv_idx,
                                                            float *__restrict__ probs, uint32_t *__restrict__ status)
 {
     extern __shared__ __align__(16) float sel_smem[];
-    select_rows<D, EPL>(g, blockIdx.y, blockIdx.x * kSelRows, sel_smem, qbar, kbarT, p, k_min, kv_cnt, kv_idx, probs,
+    select_rows<D, EPL>(g, blockIdx.y, blockIdx.x * kSelRowsFor<EPL>, sel_smem, qbar, kbarT, p, k_min, kv_cnt, kv_idx, probs,
                         status);
 }
 
@@ -676,14 +696,15 @@ static cudaError_t launch_sel_t(const Geo &g, const float *qbar, const float *kb
                                 int32_t *kv_cnt, int32_t *kv_idx, float *probs, uint32_t *status,
                                 cudaStream_t stream)
 {
-    const size_t smem = (size_t)(D + sel_slices(g.nbp) * g.nbp) * kSelRows * sizeof(float);
+    constexpr int ROWS = kSelRowsFor<EPL>;
+    const size_t smem = (size_t)(D + sel_slices(g.nbp) * g.nbp) * ROWS * sizeof(float);
     auto kern = score_select_kernel<D, EPL>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     // programmatic dependent launch: the CTAs may be scheduled while the
     // pooling kernel drains and wait in-kernel for its results
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)ceil_div(g.nb, kSelRows), (unsigned)g.BH);
+    cfg.gridDim = dim3((unsigned)ceil_div(g.nb, ROWS), (unsigned)g.BH);
     cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;

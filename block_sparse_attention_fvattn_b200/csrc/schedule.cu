@@ -9,7 +9,9 @@
 //   K3a sched_head_kernel  one CTA per head: cost of every (head, query block)
 //       unit = active 128-row query tiles x kept key/value sub-tiles (what the
 //       attention kernel executes), sorted by cost descending (ties: lower
-//       block index), plus the head's total.
+//       block index), plus the head's total. With 64-token blocks a unit is
+//       four query blocks (two pairs, one 128-row tile each) and its cost the
+//       tiles of the two pairs' unions (pair_lists_kernel builds them first).
 //   K3b sched_assign_kernel one CTA: heads sorted by total cost descending
 //       (ties: lower head), concatenated into one ranked list; rank r goes to
 //       CTA zigzag(r) (round r/C, direction alternating per round), so every
@@ -64,8 +66,86 @@ __device__ __forceinline__ int unit_tiles(const Geo &g, const int32_t *lst, int 
     return cnt * g.nsub - nlast;
 }
 
+// Paired mode (64-token blocks): pair p = query blocks (2p, 2p+1) of a head.
+// One warp merges the two kept lists into their union, ascending, each entry
+// flagged with the query blocks that keep it (kPairInA / kPairInB). The
+// attention kernel runs a pair as one 128-row query tile over the union.
+constexpr int kPairWarps = 8;
+
+__global__ void __launch_bounds__(32 * kPairWarps) pair_lists_kernel(Geo g, const int32_t *__restrict__ kv_cnt,
+                                                                     const int32_t *__restrict__ kv_idx,
+                                                                     int32_t *__restrict__ pair_cnt,
+                                                                     int32_t *__restrict__ pair_list)
+{
+    __shared__ uint32_t bm[kPairWarps][2][kMaxBlocks / 32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long pid = (long long)blockIdx.x * kPairWarps + warp;
+    if (pid >= (long long)g.BH * g.npair) return;
+    const int bh = (int)(pid / g.npair), pp = (int)(pid - (long long)bh * g.npair);
+    const int nw = (g.nb + 31) >> 5;
+    uint32_t *ma = bm[warp][0], *mb = bm[warp][1];
+    for (int w = lane; w < nw; w += 32) ma[w] = mb[w] = 0u;
+    __syncwarp();
+    for (int s = 0; s < 2; ++s) {
+        const int i = 2 * pp + s;
+        if (i >= g.nb) break;
+        const size_t u = (size_t)bh * g.nb + i;
+        const int c = min(max(__ldg(kv_cnt + u), 0), g.nb);
+        uint32_t *m = s ? mb : ma;
+        for (int e = lane; e < c; e += 32) {
+            const int j = __ldg(kv_idx + u * g.nb + e);
+            if ((unsigned)j < (unsigned)g.nb) atomicOr(&m[j >> 5], 1u << (j & 31));
+        }
+    }
+    __syncwarp();
+    // lane l writes the union's entries of bitmap word w0 + l, after those of
+    // the lower words (prefix sum of the words' counts)
+    int32_t *out = pair_list + (size_t)pid * g.nb;
+    int base = 0;
+    for (int w0 = 0; w0 < nw; w0 += 32) {
+        const int w = w0 + lane;
+        const uint32_t a = w < nw ? ma[w] : 0u, b = w < nw ? mb[w] : 0u, un = a | b;
+        const int c = __popc(un);
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        int pos = base + incl - c;
+        uint32_t rest = un;
+        while (rest) {
+            const int bit = __ffs(rest) - 1;
+            rest &= rest - 1u;
+            out[pos++] = (w * 32 + bit) | (((a >> bit) & 1u) ? kPairInA : 0) | (((b >> bit) & 1u) ? kPairInB : 0);
+        }
+        base += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+    if (lane == 0) pair_cnt[pid] = base;
+}
+
+cudaError_t launch_pair_lists(const Geo &g, const int32_t *kv_cnt, const int32_t *kv_idx, int32_t *pair_cnt,
+                              int32_t *pair_list, cudaStream_t stream)
+{
+    const long long pairs = (long long)g.BH * g.npair;
+    if (pairs == 0) return cudaSuccess;
+    pair_lists_kernel<<<(unsigned)((pairs + kPairWarps - 1) / kPairWarps), 32 * kPairWarps, 0, stream>>>(
+        g, kv_cnt, kv_idx, pair_cnt, pair_list);
+    return cudaGetLastError();
+}
+
+// Tiles of pair pp of head bh in paired mode: ceil(|union| / 2) steps of two
+// 64-token key/value blocks (0 if the pair holds no query block).
+__device__ __forceinline__ int pair_tiles(const Geo &g, int bh, int pp, const int32_t *pair_cnt, int dense)
+{
+    if (pp >= g.npair) return 0;
+    const int c = dense ? g.nb : __ldg(pair_cnt + (size_t)bh * g.npair + pp);
+    return (c + 1) >> 1;
+}
+
 __global__ void __launch_bounds__(1024) sched_head_kernel(Geo g, const int32_t *__restrict__ kv_cnt,
                                                           const int32_t *__restrict__ kv_idx, int dense,
+                                                          const int32_t *__restrict__ pair_cnt,
                                                           int32_t *__restrict__ unit_cost,
                                                           int32_t *__restrict__ head_sorted,
                                                           int64_t *__restrict__ head_cost, int npow2)
@@ -76,13 +156,18 @@ __global__ void __launch_bounds__(1024) sched_head_kernel(Geo g, const int32_t *
     const int hw = g.nbh * g.nbw;
     long long local = 0;
     for (int i = threadIdx.x; i < npow2; i += blockDim.x) {
-        if (i < g.nb) {
-            const size_t u = (size_t)bh * g.nb + i;
-            const int it = i / hw;
-            const int nh = (g.nsub == 2 && it * g.bt + g.subt < g.T) ? 2 : 1;
-            const int cnt = dense ? g.nb : __ldg(kv_cnt + u);
-            const int tiles = unit_tiles(g, dense ? nullptr : kv_idx + u * g.nb, cnt, dense);
-            const int cost = nh * tiles;
+        if (i < g.upb) {
+            const size_t u = (size_t)bh * g.upb + i;
+            int cost;
+            if (g.paired) {
+                // unit i = pairs 2i (first query tile) and 2i+1 (second)
+                cost = pair_tiles(g, bh, 2 * i, pair_cnt, dense) + pair_tiles(g, bh, 2 * i + 1, pair_cnt, dense);
+            } else {
+                const int it = i / hw;
+                const int nh = (g.nsub == 2 && it * g.bt + g.subt < g.T) ? 2 : 1;
+                const int cnt = dense ? g.nb : __ldg(kv_cnt + u);
+                cost = nh * unit_tiles(g, dense ? nullptr : kv_idx + u * g.nb, cnt, dense);
+            }
             unit_cost[u] = cost;
             local += cost;
             keys[i] = ((unsigned long long)(0xFFFFFFFFu - (uint32_t)cost) << 32) | (uint32_t)i;
@@ -99,8 +184,8 @@ __global__ void __launch_bounds__(1024) sched_head_kernel(Geo g, const int32_t *
         head_cost[bh] = s;
     }
     bitonic_sort_u64(keys, npow2);
-    for (int r = threadIdx.x; r < g.nb; r += blockDim.x)
-        head_sorted[(size_t)bh * g.nb + r] = (int32_t)(keys[r] & 0xFFFFFFFFull);
+    for (int r = threadIdx.x; r < g.upb; r += blockDim.x)
+        head_sorted[(size_t)bh * g.upb + r] = (int32_t)(keys[r] & 0xFFFFFFFFull);
 }
 
 // First index of CTA c's list when U ranks are dealt in zigzag rounds of C.
@@ -132,13 +217,13 @@ __global__ void __launch_bounds__(1024) sched_assign_kernel(Geo g, int C, const 
     for (int c = threadIdx.x; c < C; c += blockDim.x) ccost[c] = 0ull;
     __syncthreads();
     bitonic_sort_u64(hkeys, hpow2);
-    const long long U = (long long)g.BH * g.nb;
+    const long long U = (long long)g.BH * g.upb;
     for (int c = threadIdx.x; c <= C; c += blockDim.x) cta_range[c] = (int32_t)zigzag_start(c, U, C);
     for (long long r = threadIdx.x; r < U; r += blockDim.x) {
-        const long long hr = r / g.nb, local = r - hr * g.nb;
+        const long long hr = r / g.upb, local = r - hr * g.upb;
         const int head = (int)(hkeys[hr] & 0xFFFFFFFFull);
-        const int i = head_sorted[(size_t)head * g.nb + local];
-        const long long u = (long long)head * g.nb + i;
+        const int i = head_sorted[(size_t)head * g.upb + local];
+        const long long u = (long long)head * g.upb + i;
         const long long round = r / C, pos = r - round * C;
         const long long c = (round & 1) ? (C - 1 - pos) : pos;
         work[zigzag_start(c, U, C) + round] = (int32_t)u;
@@ -158,14 +243,15 @@ static int next_pow2(int n)
 
 cudaError_t launch_schedule(const Geo &g, const int32_t *kv_cnt, const int32_t *kv_idx, int dense, int num_ctas,
                             int32_t *work, int32_t *cta_range, int64_t *cta_cost, int32_t *unit_cost,
-                            int32_t *head_sorted, int64_t *head_cost, cudaStream_t stream)
+                            int32_t *head_sorted, int64_t *head_cost, const int32_t *pair_cnt,
+                            cudaStream_t stream)
 {
-    const int npow2 = next_pow2(g.nb);
+    const int npow2 = next_pow2(g.upb);
     const size_t smem_a = (size_t)npow2 * sizeof(unsigned long long);
     cudaError_t err = cudaFuncSetAttribute(sched_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a);
     if (err != cudaSuccess) return err;
-    sched_head_kernel<<<g.BH, 1024, smem_a, stream>>>(g, kv_cnt, kv_idx, dense, unit_cost, head_sorted, head_cost,
-                                                      npow2);
+    sched_head_kernel<<<g.BH, 1024, smem_a, stream>>>(g, kv_cnt, kv_idx, dense, pair_cnt, unit_cost, head_sorted,
+                                                      head_cost, npow2);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     const int hpow2 = next_pow2(g.BH);

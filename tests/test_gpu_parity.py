@@ -38,12 +38,35 @@ def _oracle_route(orc, wl, q, k):
     return g, qb, kb, r
 
 
+def _units_per_head(wl, nb):
+    bt, bh, bw = wl.block
+    return nb if bt * bh * bw == 256 else -(-nb // 4)
+
+
 def _host_costs(wl, nb, kv_cnt, kv_idx):
     """Cost of every unit as the scheduler defines it, recomputed on the host:
-    active 128-row query tiles x kept key/value sub-tiles."""
+    active 128-row query tiles x kept key/value sub-tiles. With 64-token blocks
+    a unit is query blocks 4q..4q+3: pairs (4q, 4q+1) and (4q+2, 4q+3), each
+    one 128-row tile over the union of its two lists, two blocks per step."""
     T, Hg, W = wl.grid
     bt, bh, bw = wl.block
     nbh, nbw = -(-Hg // bh), -(-W // bw)
+    BH = wl.B * wl.H
+    cnt = kv_cnt.reshape(BH, nb)
+    idx = kv_idx.reshape(BH, nb, nb)
+    if bt * bh * bw == 64:
+        upb = _units_per_head(wl, nb)
+        cost = np.zeros((BH, upb), dtype=np.int64)
+        for h in range(BH):
+            for q in range(upb):
+                for a in (4 * q, 4 * q + 2):
+                    if a >= nb:
+                        continue
+                    kept = set(idx[h, a, :cnt[h, a]].tolist())
+                    if a + 1 < nb:
+                        kept |= set(idx[h, a + 1, :cnt[h, a + 1]].tolist())
+                    cost[h, q] += (len(kept) + 1) // 2
+        return cost
     two = bt * bh * bw == 256
     subt = bt // 2 if two else bt
 
@@ -53,9 +76,6 @@ def _host_costs(wl, nb, kv_cnt, kv_idx):
 
     ns = np.array([nsub(j) for j in range(nb)])
     nh = np.array([1 + (1 if two and (i // (nbh * nbw)) * bt + subt < T else 0) for i in range(nb)])
-    BH = wl.B * wl.H
-    cnt = kv_cnt.reshape(BH, nb)
-    idx = kv_idx.reshape(BH, nb, nb)
     cost = np.zeros((BH, nb), dtype=np.int64)
     for h in range(BH):
         for i in range(nb):
@@ -111,9 +131,9 @@ def _run(wl, full_rows):
     C = eng.num_ctas
     work = eng.work.cpu().numpy()
     rng = eng.cta_range.cpu().numpy()
-    U = wl.B * wl.H * nb
+    U = wl.B * wl.H * _units_per_head(wl, nb)
     assert rng[0] == 0 and rng[C] == U and (np.diff(rng) >= 0).all()
-    assert np.array_equal(np.sort(work), np.arange(U))
+    assert np.array_equal(np.sort(work[:U]), np.arange(U))
     cost = _host_costs(wl, nb, cnt, idx)
     expect = _expected_work(cost, C)
     for c in range(C):
