@@ -143,7 +143,12 @@ FVATTN_API fvattn_status fvattn_route(const fvattn_problem *prob, const void *q,
  *
  * A work unit is one (b, h, query block i). Its cost is the number of
  * (128-row query tile, key/value sub-tile) pairs the attention kernel runs for
- * it. Units are ordered heads by total cost descending, then units within a
+ * it. With 64-token blocks the attention runs query blocks (2p, 2p+1) as one
+ * 128-row tile over the union of their two kept lists, two key blocks per
+ * step; a unit is then four query blocks 4q .. 4q+3 (two such tiles), its id
+ * u = (b*H + h)*ceil(nb/4) + q, and its cost the two tiles' steps. For that
+ * case this call also writes the unions into the workspace, where
+ * fvattn_sparse_attn reads them: give both calls the same workspace. Units are ordered heads by total cost descending, then units within a
  * head by cost descending (ties: lower index); rank r goes to CTA
  * zigzag(r) = r mod 2C < C ? r mod C : 2C-1 - r mod C, so each round of C
  * consecutive ranks (one head's units run together, which keeps its key/value
@@ -156,6 +161,7 @@ FVATTN_API fvattn_status fvattn_route(const fvattn_problem *prob, const void *q,
  *   dense           nonzero: schedule the all-blocks problem
  *   num_ctas        persistent CTAs (0 = SM count)
  *   work            out int32 [B*H*nb]    unit ids u = (b*H + h)*nb + i, grouped by CTA
+ *                                         (64-token blocks: the first B*H*ceil(nb/4) entries)
  *   cta_range       out int32 [num_ctas+1] CTA c runs work[cta_range[c] .. cta_range[c+1])
  *   cta_cost        out int64 [num_ctas]  predicted cost per CTA, or NULL
  */
@@ -172,14 +178,18 @@ FVATTN_API fvattn_status fvattn_schedule(const fvattn_problem *prob, const int32
  *
  * For every valid query token r of block i: o_r = sum over the valid tokens k
  * of the blocks in S_i of softmax_k(scale * q_r . k_k) * v_k, computed with an
- * online softmax over 128-token (64 for 64-token blocks) key/value sub-tiles.
+ * online softmax over 128-token key/value tiles (64-token blocks: two key
+ * blocks per tile, shared by two query blocks, each of which masks the key
+ * blocks it did not keep).
  * dense != 0 uses every block (the VSA_ALL_BLOCKS route, section 3/5), giving
  * the in-library dense comparison.
  *
  *   q, k, v        bf16 [B,H,N,D]
  *   kv_cnt, kv_idx lists from fvattn_route (ignored if dense)
- *   work, cta_range from fvattn_schedule with the same num_ctas and dense flag
- *                  (both NULL: units in index order). The CTAs take ranks
+ *   work, cta_range from fvattn_schedule with the same num_ctas, dense flag
+ *                  and workspace (both NULL: units in index order; with
+ *                  64-token blocks the call then builds the pair unions in the
+ *                  workspace itself, one extra kernel). The CTAs take ranks
  *                  0, 1, 2, ... of the scheduler's longest-first order from a
  *                  counter shared through the workspace (rank r is entry
  *                  r / num_ctas of list zigzag(r)), so a CTA that finishes early
