@@ -25,13 +25,13 @@
 // article, section 5.1, on n x n masks at ~400k tokens).
 //
 // Roles (384 threads = 3 warpgroups, one CTA per SM):
-//   warp 0      TMA producer: Q halves, K and V sub-tiles into rings
+//   warp 0      TMA producer of Q halves and K sub-tiles; takes the units
 //   warp 1      QK issuer (one thread) and owner of the TMEM allocation:
 //               S = Q_h K^T (A and B from shared memory)
 //   warp 2      PV issuer (one thread): O_h += P_h V (A = P_h from TMEM,
 //               B = V from shared memory, MN-major). Two issuing threads keep
 //               the tensor core fed while either one waits on a barrier.
-//   warp 3      idle (it only returns registers)
+//   warp 3      TMA producer of V sub-tiles (follows warp 0's units)
 //   warps 4-7   softmax + epilogue for query half 0
 //   warps 8-11  softmax + epilogue for query half 1
 // A warp reaches TMEM lanes 32*(warp % 4) .. +31, so each softmax warpgroup
@@ -59,8 +59,6 @@
 
 namespace fvattn {
 
-constexpr int kNK = 2;  // K ring stages
-constexpr int kNV = 3;  // V ring stages
 constexpr int kUnitSlots = 4;  // ring of unit ids handed from the producer to the other roles
 constexpr int kThreads = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -78,6 +76,11 @@ struct RegSplit {
 
 template <int D, int BKV, bool PAIRED = false>
 struct AttnLayout {
+    // Ring stages: a V tile waits for a softmax before its product, so V gets
+    // the deeper ring (measured on B200; paired mode with 3 K / 2 V stages
+    // ran 8% slower)
+    static constexpr int kNK = 2;  // K ring stages
+    static constexpr int kNV = 3;  // V ring stages
     static constexpr int kDH = D / 64;              // 128-byte column slabs per row
     static constexpr int kQSlab = 128 * 128;        // bytes of one 128-row slab
     static constexpr int kKVSlab = BKV * 128;
@@ -98,8 +101,9 @@ struct AttnLayout {
                          bVEmpty = bVFull + kNV, bSFull = bVEmpty + kNV, bSFree = bSFull + 2, bPFull = bSFree + 1,
                          bPFree = bPFull + 2, bOFull = bPFree + 2, bOEmpty = bOFull + 2, bDrain = bOEmpty + 2,
                          bUFull = bDrain + 2, bUEmpty = bUFull + kUnitSlots, kNumBars = bUEmpty + kUnitSlots;
-    // arrivals that free a unit slot: QK issuer, PV issuer and the 8 softmax warps
-    static constexpr int kUnitConsumers = 10;
+    // arrivals that free a unit slot: the V producer, the QK and PV issuers and
+    // the 8 softmax warps
+    static constexpr int kUnitConsumers = 11;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 64;
     static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
@@ -214,6 +218,7 @@ __device__ __forceinline__ PairUnit load_pair_unit(const Geo &g, int u, const in
 // columns are masked out for every row.
 __device__ __forceinline__ int pair_entry(const int32_t *lst, int c, int e)
 {
+    if (c <= 0) return 0;  // empty half: never used
     const bool past = e >= c;
     const int ee = past ? c - 1 : e;
     const int v = lst ? __ldg(lst + ee) : (ee | kPairInA | kPairInB);
@@ -351,143 +356,132 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t q_bytes = (uint32_t)L::kDH * (uint32_t)g.rows * 128u;
 
     if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(RegSplit<D, BKV>::kLow));
-    if (warp == 0) {
-        // ================= TMA producer =================
+    if (warp == 0 || warp == 3) {
+        // ================= TMA producers =================
+        // warp 0 takes the units and loads Q and K; warp 3 follows the same
+        // units (through the unit ring) and loads V, so a K load never waits
+        // for a V slot, which frees only after a softmax and a PV
         if (lane == 0) {
-            tma_prefetch_desc(&tm_q);
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
+            const bool vrole = warp == 3;
+            if (vrole) {
+                tma_prefetch_desc(&tm_v);
+            } else {
+                tma_prefetch_desc(&tm_q);
+                tma_prefetch_desc(&tm_k);
+            }
             int kc = 0, vc = 0;
             uint32_t q_par = 0, q_used = 0;  // per half: loads issued & 1, any load issued
             bool ok = true;
-            for (int n = 0; ok; ++n) {
-                const int slot = n % kUnitSlots;
-                if (n >= kUnitSlots &&
-                    !mbar_wait(bar(L::bUEmpty + slot), (uint32_t)((n / kUnitSlots) - 1) & 1u, abort_flag)) {
-                    ok = false;
-                    break;
+            // one key/value tile: blocks j0 (rows 0..) and, paired, j1 (rows 64..)
+            auto load_kv = [&](int j0, int j1, int t_off, int ubh) -> bool {
+                const bool pair = PAIRED;
+                if (!vrole) {
+                    const int ks = kc % L::kNK;
+                    if (kc >= L::kNK && !mbar_wait(bar(L::bKEmpty + ks), ((kc / L::kNK) - 1) & 1, abort_flag))
+                        return false;
+                    mbar_arrive_expect_tx(bar(L::bKFull + ks), kTileBytes);
+                    for (int s2 = 0; s2 < (pair ? 2 : 1); ++s2) {
+                        int jt, jy, jx;
+                        block_coords(g, s2 ? j1 : j0, jt, jy, jx);
+                        for (int dh = 0; dh < L::kDH; ++dh)
+                            tma_load_5d(sbase + L::kK + (ks * L::kDH + dh) * L::kKVSlab + s2 * kHalfRows, &tm_k,
+                                        bar(L::bKFull + ks), dh * 64, jx * g.bw, jy * g.bh, jt * g.bt + t_off, ubh);
+                    }
+                    ++kc;
+                } else {
+                    const int vs = vc % L::kNV;
+                    if (vc >= L::kNV && !mbar_wait(bar(L::bVEmpty + vs), ((vc / L::kNV) - 1) & 1, abort_flag))
+                        return false;
+                    mbar_arrive_expect_tx(bar(L::bVFull + vs), kTileBytes);
+                    for (int s2 = 0; s2 < (pair ? 2 : 1); ++s2) {
+                        int jt, jy, jx;
+                        block_coords(g, s2 ? j1 : j0, jt, jy, jx);
+                        for (int dh = 0; dh < L::kDH; ++dh)
+                            tma_load_5d(sbase + L::kV + (vs * L::kDH + dh) * L::kKVSlab + s2 * kHalfRows, &tm_v,
+                                        bar(L::bVFull + vs), dh * 64, jx * g.bw, jy * g.bh, jt * g.bt + t_off, ubh);
+                    }
+                    ++vc;
                 }
-                const long long r = (long long)atomicAdd(unit_cursor, 1u);
-                const int u = r < n_units ? rank_to_unit(r, work, cta_range) : -1;
-                unit_slots[slot] = u;
-                mbar_arrive(bar(L::bUFull + slot));  // release: the id is visible to the waiting roles
+                return true;
+            };
+            // Q half h: rows 0.. from block i0 at frame offset t_off, paired also rows 64.. from i0+1
+            auto load_q = [&](int h, int i0, int nblk, int t_off, int ubh) -> bool {
+                if (((q_used >> h) & 1u) && !mbar_wait(bar(L::bQEmpty + h), ((q_par >> h) & 1u) ^ 1u, abort_flag))
+                    return false;
+                mbar_arrive_expect_tx(bar(L::bQFull + h), PAIRED ? (uint32_t)nblk * L::kDH * kHalfRows : q_bytes);
+                for (int s2 = 0; s2 < nblk; ++s2) {
+                    int jt, jy, jx;
+                    block_coords(g, i0 + s2, jt, jy, jx);
+                    for (int dh = 0; dh < L::kDH; ++dh)
+                        tma_load_5d(sbase + L::kQ + (h * L::kDH + dh) * L::kQSlab + s2 * kHalfRows, &tm_q,
+                                    bar(L::bQFull + h), dh * 64, jx * g.bw, jy * g.bh, jt * g.bt + t_off, ubh);
+                }
+                q_par ^= 1u << h;
+                q_used |= 1u << h;
+                return true;
+            };
+            for (int n = 0; ok; ++n) {
+                int u;
+                if (!vrole) {
+                    const int slot = n % kUnitSlots;
+                    if (n >= kUnitSlots &&
+                        !mbar_wait(bar(L::bUEmpty + slot), (uint32_t)((n / kUnitSlots) - 1) & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const long long r = (long long)atomicAdd(unit_cursor, 1u);
+                    u = r < n_units ? rank_to_unit(r, work, cta_range) : -1;
+                    unit_slots[slot] = u;
+                    mbar_arrive(bar(L::bUFull + slot));  // release: the id is visible to the waiting roles
+                } else {
+                    int slot;
+                    u = feed.next(abort_flag, ok, slot);
+                    if (!ok) break;
+                    mbar_arrive(bar(L::bUEmpty + slot));
+                }
                 if (u < 0) break;
                 if constexpr (PAIRED) {
                     const PairUnit P = load_pair_unit(g, u, pair_cnt, pair_list, dense);
-                    for (int h = 0; h < 2 && ok; ++h) {
+                    for (int h = 0; h < 2 && ok && !vrole; ++h) {
                         if (P.cnt(h) == 0) continue;
-                        if (((q_used >> h) & 1u) &&
-                            !mbar_wait(bar(L::bQEmpty + h), ((q_par >> h) & 1u) ^ 1u, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
                         const int qa = 2 * (2 * P.q + h);  // rows 0-63: block qa, rows 64-127: block qa+1
-                        const int nq = qa + 1 < g.nb ? 2 : 1;
-                        mbar_arrive_expect_tx(bar(L::bQFull + h), (uint32_t)nq * L::kDH * kHalfRows);
-                        for (int s2 = 0; s2 < nq; ++s2) {
-                            int jt, jy, jx;
-                            block_coords(g, qa + s2, jt, jy, jx);
-                            for (int dh = 0; dh < L::kDH; ++dh)
-                                tma_load_5d(sbase + L::kQ + (h * L::kDH + dh) * L::kQSlab + s2 * kHalfRows, &tm_q,
-                                            bar(L::bQFull + h), dh * 64, jx * g.bw, jy * g.bh, jt * g.bt, P.bh);
-                        }
-                        q_par ^= 1u << h;
-                        q_used |= 1u << h;
+                        ok = load_q(h, qa, qa + 1 < g.nb ? 2 : 1, 0, P.bh);
                     }
                     // key/value tiles, the two halves interleaved: round r is tile r of
                     // half 0, then tile r of half 1 (each while that half has one)
                     const int rounds = max(P.tiles(0), P.tiles(1));
+                    // a round's four entries are loaded one round ahead
+                    int cur[4] = {pair_entry(P.l0, P.c0, 0), pair_entry(P.l0, P.c0, 1), pair_entry(P.l1, P.c1, 0),
+                                  pair_entry(P.l1, P.c1, 1)};
                     for (int r = 0; r < rounds && ok; ++r) {
+                        const int nxt[4] = {pair_entry(P.l0, P.c0, 2 * r + 2), pair_entry(P.l0, P.c0, 2 * r + 3),
+                                            pair_entry(P.l1, P.c1, 2 * r + 2), pair_entry(P.l1, P.c1, 2 * r + 3)};
                         for (int h = 0; h < 2 && ok; ++h) {
                             if (r >= P.tiles(h)) continue;
-                            const int jb[2] = {pair_entry(P.list(h), P.cnt(h), 2 * r) & kPairBlockMask,
-                                               pair_entry(P.list(h), P.cnt(h), 2 * r + 1) & kPairBlockMask};
-                            const int ks = kc % kNK;
-                            if (kc >= kNK && !mbar_wait(bar(L::bKEmpty + ks), ((kc / kNK) - 1) & 1, abort_flag)) {
-                                ok = false;
-                                break;
-                            }
-                            mbar_arrive_expect_tx(bar(L::bKFull + ks), kTileBytes);
-                            for (int s2 = 0; s2 < 2; ++s2) {
-                                int jt, jy, jx;
-                                block_coords(g, jb[s2], jt, jy, jx);
-                                for (int dh = 0; dh < L::kDH; ++dh)
-                                    tma_load_5d(sbase + L::kK + (ks * L::kDH + dh) * L::kKVSlab + s2 * kHalfRows,
-                                                &tm_k, bar(L::bKFull + ks), dh * 64, jx * g.bw, jy * g.bh,
-                                                jt * g.bt, P.bh);
-                            }
-                            ++kc;
-                            const int vs = vc % kNV;
-                            if (vc >= kNV && !mbar_wait(bar(L::bVEmpty + vs), ((vc / kNV) - 1) & 1, abort_flag)) {
-                                ok = false;
-                                break;
-                            }
-                            mbar_arrive_expect_tx(bar(L::bVFull + vs), kTileBytes);
-                            for (int s2 = 0; s2 < 2; ++s2) {
-                                int jt, jy, jx;
-                                block_coords(g, jb[s2], jt, jy, jx);
-                                for (int dh = 0; dh < L::kDH; ++dh)
-                                    tma_load_5d(sbase + L::kV + (vs * L::kDH + dh) * L::kKVSlab + s2 * kHalfRows,
-                                                &tm_v, bar(L::bVFull + vs), dh * 64, jx * g.bw, jy * g.bh,
-                                                jt * g.bt, P.bh);
-                            }
-                            ++vc;
+                            ok = load_kv((h ? cur[2] : cur[0]) & kPairBlockMask, (h ? cur[3] : cur[1]) & kPairBlockMask,
+                                         0, P.bh);
                         }
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) cur[x] = nxt[x];
                     }
                     continue;
                 }
                 const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
-                const int x0 = U.ix * g.bw, y0 = U.iy * g.bh, t0 = U.it * g.bt;
-                for (int h = 0; h < U.nh && ok; ++h) {
-                    if (((q_used >> h) & 1u) &&
-                        !mbar_wait(bar(L::bQEmpty + h), ((q_par >> h) & 1u) ^ 1u, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(bar(L::bQFull + h), q_bytes);
-                    for (int dh = 0; dh < L::kDH; ++dh)
-                        tma_load_5d(sbase + L::kQ + (h * L::kDH + dh) * L::kQSlab, &tm_q, bar(L::bQFull + h),
-                                    dh * 64, x0, y0, t0 + h * g.subt, U.bh);
-                    q_par ^= 1u << h;
-                    q_used |= 1u << h;
-                }
+                for (int h = 0; h < U.nh && ok && !vrole; ++h) ok = load_q(h, U.i, 1, h * g.subt, U.bh);
                 TileCursor cur;
                 for (int k = 0; k < U.nkv && ok; ++k) {
-                    const int j = cur.block(U);
-                    int jt, jy, jx;
-                    block_coords(g, j, jt, jy, jx);
-                    const int tt0 = jt * g.bt + cur.s * g.subt;
-                    const int ks = kc % kNK;
-                    if (kc >= kNK && !mbar_wait(bar(L::bKEmpty + ks), ((kc / kNK) - 1) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(bar(L::bKFull + ks), kTileBytes);
-                    for (int dh = 0; dh < L::kDH; ++dh)
-                        tma_load_5d(sbase + L::kK + (ks * L::kDH + dh) * L::kKVSlab, &tm_k, bar(L::bKFull + ks),
-                                    dh * 64, jx * g.bw, jy * g.bh, tt0, U.bh);
-                    ++kc;
-                    const int vs = vc % kNV;
-                    if (vc >= kNV && !mbar_wait(bar(L::bVEmpty + vs), ((vc / kNV) - 1) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(bar(L::bVFull + vs), kTileBytes);
-                    for (int dh = 0; dh < L::kDH; ++dh)
-                        tma_load_5d(sbase + L::kV + (vs * L::kDH + dh) * L::kKVSlab, &tm_v, bar(L::bVFull + vs),
-                                    dh * 64, jx * g.bw, jy * g.bh, tt0, U.bh);
-                    ++vc;
+                    ok = load_kv(cur.block(U), 0, cur.s * g.subt, U.bh);
                     cur.advance(g, U);
                 }
             }
             if (!ok) {
                 // wind down: let every copy already issued land before the CTA exits
-                for (int s = 0; s < kNK; ++s) {
-                    const int n = (kc > s) ? (kc - s + kNK - 1) / kNK : 0;
+                for (int s = 0; s < L::kNK; ++s) {
+                    const int n = (kc > s) ? (kc - s + L::kNK - 1) / L::kNK : 0;
                     if (n > 0) mbar_wait_for(bar(L::bKFull + s), (n - 1) & 1, 50000000ull);
                 }
-                for (int s = 0; s < kNV; ++s) {
-                    const int n = (vc > s) ? (vc - s + kNV - 1) / kNV : 0;
+                for (int s = 0; s < L::kNV; ++s) {
+                    const int n = (vc > s) ? (vc - s + L::kNV - 1) / L::kNV : 0;
                     if (n > 0) mbar_wait_for(bar(L::bVFull + s), (n - 1) & 1, 50000000ull);
                 }
                 for (int h = 0; h < 2; ++h)
@@ -533,8 +527,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int r = 0; r < rounds && ok; ++r) {
                         for (int h = 0; h < 2 && ok; ++h) {
                             if (r >= P.tiles(h)) continue;
-                            const int ks = kc % kNK;
-                            if (!mbar_wait(bar(L::bKFull + ks), (kc / kNK) & 1, abort_flag)) { ok = false; break; }
+                            const int ks = kc % L::kNK;
+                            if (!mbar_wait(bar(L::bKFull + ks), (kc / L::kNK) & 1, abort_flag)) { ok = false; break; }
                             if (qk_count > 0 && !mbar_wait(bar(L::bSFree), (qk_count - 1) & 1, abort_flag)) {
                                 ok = false;
                                 break;
@@ -556,8 +550,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ph_q ^= 1u << h;
                 }
                 for (int k = 0; k < U.nkv && ok; ++k) {
-                    const int ks = kc % kNK;
-                    if (!mbar_wait(bar(L::bKFull + ks), (kc / kNK) & 1, abort_flag)) { ok = false; break; }
+                    const int ks = kc % L::kNK;
+                    if (!mbar_wait(bar(L::bKFull + ks), (kc / L::kNK) & 1, abort_flag)) { ok = false; break; }
                     for (int h = 0; h < U.nh; ++h) {
                         // S is shared: overwrite it only once the previous S has been
                         // copied into registers by its softmax warpgroup
@@ -619,8 +613,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int r = 0; r < rounds && ok; ++r) {
                         for (int h = 0; h < 2 && ok; ++h) {
                             if (r >= P.tiles(h)) continue;
-                            const int vs = vc % kNV;
-                            if (!mbar_wait(bar(L::bVFull + vs), (vc / kNV) & 1, abort_flag)) { ok = false; break; }
+                            const int vs = vc % L::kNV;
+                            if (!mbar_wait(bar(L::bVFull + vs), (vc / L::kNV) & 1, abort_flag)) { ok = false; break; }
                             ok = mbar_wait(bar(L::bPFull + h), (ph_p >> h) & 1u, abort_flag);
                             ph_p ^= 1u << h;
                             if (ok && r == 0) ok = o_free(h);
@@ -640,8 +634,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
                 for (int k = 0; k < U.nkv && ok; ++k) {
-                    const int vs = vc % kNV;
-                    if (!mbar_wait(bar(L::bVFull + vs), (vc / kNV) & 1, abort_flag)) { ok = false; break; }
+                    const int vs = vc % L::kNV;
+                    if (!mbar_wait(bar(L::bVFull + vs), (vc / L::kNV) & 1, abort_flag)) { ok = false; break; }
                     for (int h = 0; h < U.nh; ++h) {
                         ok = mbar_wait(bar(L::bPFull + h), (ph_p >> h) & 1u, abort_flag);
                         ph_p ^= 1u << h;
