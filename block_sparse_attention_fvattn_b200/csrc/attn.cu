@@ -677,7 +677,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         float m = -INFINITY, l = 0.f;
         // One key/value tile of this half: S from TMEM, masks, online softmax,
         // P into TMEM (after the previous PV of this half), lazy O rescale.
-        auto tile = [&](bool first, auto &&apply_mask) -> bool {
+        // keep: bit 0 / bit 1 = columns 0-63 / 64-127 take part (paired mode:
+        // the key block there was kept by this row's query block); apply_mask
+        // masks padding inside kept columns.
+        auto tile = [&](bool first, uint32_t keep, auto &&apply_mask) -> bool {
             if (!mbar_wait(bar(L::bSFull + h), sf & 1, abort_flag)) return false;
             ++sf;
             tc_fence_after();
@@ -696,15 +699,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < BKV; ++c) x[c] = __uint_as_float(r[c]);
             apply_mask(x);
-            // row maximum: 8 independent chains of three-input max, then a tree
+            // row maximum of each 64-column half: 4 independent chains of
+            // three-input max each, then trees; a half that takes no part is left out
             float m8[8];
 #pragma unroll
             for (int q8 = 0; q8 < 8; ++q8) m8[q8] = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < BKV; c += 16)
+            for (int c = 0; c < BKV / 2; c += 8)
 #pragma unroll
-                for (int q8 = 0; q8 < 8; ++q8) m8[q8] = max3f(m8[q8], x[c + 2 * q8], x[c + 2 * q8 + 1]);
-            const float mx = fmaxf(max3f(m8[0], m8[1], m8[2]), max3f(max3f(m8[3], m8[4], m8[5]), m8[6], m8[7]));
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    m8[q4] = max3f(m8[q4], x[c + 2 * q4], x[c + 2 * q4 + 1]);
+                    m8[4 + q4] = max3f(m8[4 + q4], x[BKV / 2 + c + 2 * q4], x[BKV / 2 + c + 2 * q4 + 1]);
+                }
+            const float mxa = fmaxf(max3f(m8[0], m8[1], m8[2]), m8[3]);
+            const float mxb = fmaxf(max3f(m8[4], m8[5], m8[6]), m8[7]);
+            const float mx = fmaxf((keep & 1u) ? mxa : -INFINITY, (keep & 2u) ? mxb : -INFINITY);
             const float mt = mx * sl2;
             float alpha = 1.0f;
             bool rescale = false;
@@ -725,12 +734,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             // paired mode: a row whose own query block kept no block of the
             // tiles so far has m = -inf; its p are 0 (not inf - inf)
             const float m_use = (PAIRED && m == -INFINITY) ? 0.f : m;
-            const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_use, -m_use);
+            // a half that takes no part gets 2^-inf = 0
+            const float na = (keep & 1u) ? -m_use : -INFINITY, nb = (keep & 2u) ? -m_use : -INFINITY;
+            const uint64_t sl2x2 = f2_pack(sl2, sl2), neg_a = f2_pack(na, na), neg_b = f2_pack(nb, nb);
             uint64_t s4[4] = {0ull, 0ull, 0ull, 0ull};
             uint32_t pk[BKV / 2];
 #pragma unroll
             for (int q2 = 0; q2 < BKV / 2; ++q2) {
-                const uint64_t a = f2_fma(f2_pack(x[2 * q2], x[2 * q2 + 1]), sl2x2, negm2);
+                const uint64_t a = f2_fma(f2_pack(x[2 * q2], x[2 * q2 + 1]), sl2x2, q2 < BKV / 4 ? neg_a : neg_b);
                 float p0, p1;
                 if ((q2 & 7) < FV_POLY_PAIRS / 2) {
                     exp2_poly_x2(a, p0, p1);
@@ -830,9 +841,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int r = 0; r < n_h; ++r) {
                     // the next tile's entries are loaded now and used next iteration
                     const int nxt0 = pair_entry(lst, c_h, 2 * r + 2), nxt1 = pair_entry(lst, c_h, 2 * r + 3);
-                    // column word w covers key block ent(w/2): all masked unless this
-                    // row's query block kept it, then its padding masked
-                    uint32_t mw[4];
+                    // columns [64*s2, 64*s2+64) hold key block ent(s2): they take part
+                    // if this row's query block kept it, with its padding masked
+                    uint32_t keep = 0, mw[4];
                     bool all = true;
 #pragma unroll
                     for (int s2 = 0; s2 < 2; ++s2) {
@@ -841,15 +852,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         block_coords(g, ent & kPairBlockMask, jt, jy, jx);
                         const int wv = min(g.bw, g.W - jx * g.bw), hv = min(g.bh, g.Hg - jy * g.bh);
                         const int tv = min(g.bt, g.T - jt * g.bt);
-                        const bool keep = (ent & keeper) != 0;
+                        const bool kept = (ent & keeper) != 0;
                         const bool full = wv == g.bw && hv == g.bh && tv == g.bt;
+                        keep |= kept ? (1u << s2) : 0u;
 #pragma unroll
                         for (int w = 0; w < L::kMaskWords; ++w) {
-                            const uint32_t word = !keep ? 0u
-                                                  : full ? 0xFFFFFFFFu
-                                                         : (mask_w[(wv - 1) * L::kMaskWords + w] &
-                                                            mask_h[(hv - 1) * L::kMaskWords + w] &
-                                                            mask_t[(tv - 1) * L::kMaskWords + w]);
+                            const uint32_t word = (!kept || full) ? 0xFFFFFFFFu
+                                                                  : (mask_w[(wv - 1) * L::kMaskWords + w] &
+                                                                     mask_h[(hv - 1) * L::kMaskWords + w] &
+                                                                     mask_t[(tv - 1) * L::kMaskWords + w]);
                             mw[s2 * L::kMaskWords + w] = word;
                             all = all && word == 0xFFFFFFFFu;
                         }
@@ -862,7 +873,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int b = 0; b < 32; ++b)
                                 if (!((mw[w] >> b) & 1u)) x[w * 32 + b] = -INFINITY;
                     };
-                    if (!tile(r == 0, mask)) { ok = false; break; }
+                    if (!tile(r == 0, keep, mask)) { ok = false; break; }
                     ent0 = nxt0;
                     ent1 = nxt1;
                 }
@@ -899,7 +910,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 };
-                if (!tile(k == 0, mask)) { ok = false; break; }
+                if (!tile(k == 0, 3u, mask)) { ok = false; break; }
                 if (g.nsub == 2 && s_sub == 0 && jt * g.bt + g.subt < g.T) {
                     s_sub = 1;
                 } else {
