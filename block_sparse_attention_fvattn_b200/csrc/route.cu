@@ -214,6 +214,15 @@ __device__ __forceinline__ float key_float(uint32_t key)
     return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
+// Unnormalised softmax weight exp(s - mx) of a score, as 2^((s - mx) log2 e)
+// on the hardware exp2 (relative error ~1e-6 here, far inside the 1e-5 Top-p
+// window). Every mass of a row is computed by this one expression, so a
+// block's weight is bit-identical wherever it is recomputed from its key.
+__device__ __forceinline__ float row_weight(float s, float mx)
+{
+    return ex2_approx((s - mx) * 1.4426950408889634f);
+}
+
 // Bitonic sort, descending, of the 32*EPL keys a warp holds: lane l holds
 // positions l*EPL .. l*EPL+EPL-1. Exchanges between positions closer than
 // EPL stay in a lane's registers; the others go through shuffles.
@@ -283,7 +292,8 @@ __device__ __forceinline__ float mass_at_least(const uint32_t (&key)[EPL], const
 {
     float m[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) m[e & 3] += (key[e] >= t) ? pv(e) : 0.f;
+    for (int e = 0; e < EPL; ++e)
+        if (key[e] >= t) m[e & 3] += pv(e);
     return warp_sum((m[0] + m[1]) + (m[2] + m[3]));
 }
 
@@ -367,7 +377,7 @@ __device__ __forceinline__ void window_boundary(const uint32_t (&key)[EPL], cons
     warp_sort_desc<1>(ck, lane);
     int nk;  // kept candidates: a prefix of the sorted ones
     if constexpr (MASS) {
-        const float cp = ck[0] ? expf(key_float(ck[0]) - mx) : 0.f;  // the same value as pv of that block
+        const float cp = ck[0] ? row_weight(key_float(ck[0]), mx) : 0.f;  // the same value as pv of that block
         float incl = cp;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -551,7 +561,7 @@ __device__ __forceinline__ void select_rows(const Geo &g, int bh, int i0, float 
 #pragma unroll
             for (int e = 0; e < EPL; ++e) {
                 c[e] = run;  // mass before this position, within the lane
-                run += sk[e] ? expf(key_float(sk[e]) - mx) : 0.f;
+                run += sk[e] ? row_weight(key_float(sk[e]), mx) : 0.f;
             }
             float incl = run;
 #pragma unroll
@@ -588,7 +598,7 @@ __device__ __forceinline__ void select_rows(const Geo &g, int bh, int i0, float 
             for (int e = 0; e < EPL; ++e) {
                 const int j = lane + 32 * e;
                 if (j < nb) {
-                    const float pj = expf(key_float(key[e]) - mx);
+                    const float pj = row_weight(key_float(key[e]), mx);
                     srow[j] = pj;
                     kmin = min(kmin, key[e]);
                     kmax = max(kmax, key[e]);
@@ -596,7 +606,9 @@ __device__ __forceinline__ void select_rows(const Geo &g, int bh, int i0, float 
                 }
             }
             const float *pvr = srow;  // pv of block j at pvr[j]; read only where key[e] != 0
-            auto pv = [&](int e) { return key[e] ? pvr[lane + 32 * e] : 0.f; };
+            // read only under a key test that fails for the padding keys (0); the
+            // shared memory is padded so those reads stay inside it
+            auto pv = [&](int e) { return pvr[lane + 32 * e]; };
             z = warp_sum((zl[0] + zl[1]) + (zl[2] + zl[3]));
             kmin = warp_min_u(kmin);
             kmax = warp_max_u(kmax);
@@ -635,7 +647,7 @@ __device__ __forceinline__ void select_rows(const Geo &g, int bh, int i0, float 
             base += __popc(sm);
             if (probs && valid) {
                 float pj;
-                if constexpr (kSortedSelect<EPL>) pj = expf(key_float(key[e]) - mx);
+                if constexpr (kSortedSelect<EPL>) pj = row_weight(key_float(key[e]), mx);
                 else pj = srow[j];
                 probs[row * nb + j] = pj * invz;
             }
@@ -697,7 +709,8 @@ static cudaError_t launch_sel_t(const Geo &g, const float *qbar, const float *kb
                                 cudaStream_t stream)
 {
     constexpr int ROWS = kSelRowsFor<EPL>;
-    const size_t smem = (size_t)(D + sel_slices(g.nbp) * g.nbp) * ROWS * sizeof(float);
+    // + 32*EPL floats: a row's lanes read positions up to 32*EPL - 1
+    const size_t smem = ((size_t)(D + sel_slices(g.nbp) * g.nbp) * ROWS + 32 * EPL) * sizeof(float);
     auto kern = score_select_kernel<D, EPL>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
