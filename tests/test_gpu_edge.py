@@ -113,6 +113,30 @@ def test_output_independent_of_cta_count(num_ctas):
     assert torch.equal(out, ref)
 
 
+@pytest.mark.parametrize("num_ctas", [1, 5, 148])
+def test_paired_output_independent_of_cta_count_and_schedule(num_ctas):
+    # 64-token blocks run as paired units; the result must not depend on the
+    # CTA count, nor on whether work lists come from fvattn_schedule or the
+    # call builds the pair unions itself (units in index order)
+    from block_sparse_attention_fvattn_b200 import fvattn as fa
+    wl = gen.custom("paired_ctas", 1, 3, 128, (8, 12, 20), (4, 4, 4), 0.9, 3, sigma=2.0, a_range=(0.5, 4.0),
+                    seed=38)
+    q, k, v = fvtest.make_on_gpu(wl)
+    ref = _engine(wl, num_ctas=148)(q, k, v).clone()
+    eng = _engine(wl, num_ctas=num_ctas)
+    out = eng(q, k, v)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    # no work lists: a fresh workspace, so the pair unions must come from this call
+    ws = torch.zeros_like(eng.ws)
+    fa.workspace_init(ws)
+    out2 = torch.zeros_like(q)
+    fa.sparse_attn(eng.geo, q, k, v, eng.kv_cnt, eng.kv_idx, None, None, num_ctas, False, out2, ws)
+    torch.cuda.synchronize()
+    assert fa.read_device_status(ws) == 0
+    assert torch.equal(out2, ref)
+
+
 def test_repeatable():
     wl = gen.WORKLOADS["wan5b"]
     q, k, v = fvtest.make_on_gpu(wl)

@@ -27,6 +27,9 @@ SMALL = [
     gen.custom("blk64_ragged_d64", 1, 2, 64, (6, 10, 9), (4, 4, 4), 0.9, 3, sigma=1.5, a_range=(0.5, 4.0),
                seed=25),
     gen.custom("iid_tiny", 1, 2, 64, (8, 16, 16), (4, 8, 8), 0.9, 2, seed=26),
+    # 15 64-token blocks: the last pair holds one query block, the last unit one and a half pairs
+    gen.custom("blk64_odd_pairs", 2, 2, 128, (4, 12, 20), (4, 4, 4), 0.8, 2, sigma=1.5, a_range=(0.5, 4.0),
+               seed=27),
 ]
 FULL = [gen.WORKLOADS[n] for n in gen.WORKLOAD_ORDER]
 
