@@ -303,7 +303,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto bar = [&](int idx) -> uint32_t { return sbase + L::kBar + 8u * (uint32_t)idx; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint64_t t_start = globaltimer_ns();
 
     // ---- set-up: per-axis column masks, barriers, TMEM
     {
@@ -342,6 +341,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // launched as a programmatic dependent of the scheduler: everything above
+    // overlaps its tail; lists, work and counters are read only after this
+    pdl_wait();
+    const uint64_t t_start = globaltimer_ns();
 
     // Units are taken dynamically, longest first, from a counter shared by all
     // CTAs (workspace header word 1); the producer thread takes them and hands
@@ -994,9 +997,8 @@ static cudaError_t launch_attn_t(const Geo &g, const CUtensorMap &mq, const CUte
         return cudaErrorInvalidConfiguration;
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (err != cudaSuccess) return err;
-    kern<<<grid, kThreads, L::kAlloc, stream>>>(mq, mk, mv, g, kv_cnt, kv_idx, pair_cnt, pair_list, work, cta_range,
-                                                dense, (__nv_bfloat16 *)out, cta_ns, status);
-    return cudaGetLastError();
+    return launch_dependent(kern, dim3(grid), dim3(kThreads), L::kAlloc, stream, mq, mk, mv, g, kv_cnt, kv_idx,
+                            pair_cnt, pair_list, work, cta_range, dense, (__nv_bfloat16 *)out, cta_ns, status);
 }
 
 cudaError_t launch_attn(const Geo &g, const void *q, const void *k, const void *v, const int32_t *kv_cnt,

@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geo g, int nxs, cons
     }
     // every load of this CTA has been consumed: the selection kernel, if it
     // was launched as a programmatic dependent, may begin its launch
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    pdl_release();
 
 #pragma unroll
     for (int s = 0; s < NS; ++s) {
@@ -485,8 +485,10 @@ __device__ __forceinline__ void select_rows(const Geo &g, int bh, int i0, float 
     const int nrow = min(ROWS, g.nb - i0);
     const int nbp = g.nbp;
 
-    // launched as a programmatic dependent of the pooling kernel: wait for it
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // launched as a programmatic dependent of the pooling kernel: let the
+    // scheduler launch behind this grid, then wait for the pooled means
+    pdl_release();
+    pdl_wait();
     for (int idx = threadIdx.x; idx < ROWS * D; idx += blockDim.x) {
         const int r = idx / D, d = idx - r * D;
         qsT[d * ROWS + r] = (r < nrow) ? qbar[((size_t)bh * g.nb + i0 + r) * D + d] : 0.f;
@@ -716,17 +718,8 @@ static cudaError_t launch_sel_t(const Geo &g, const float *qbar, const float *kb
     if (err != cudaSuccess) return err;
     // programmatic dependent launch: the CTAs may be scheduled while the
     // pooling kernel drains and wait in-kernel for its results
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)ceil_div(g.nb, ROWS), (unsigned)g.BH);
-    cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, g, qbar, kbarT, p, k_min, kv_cnt, kv_idx, probs, status);
+    return launch_dependent(kern, dim3((unsigned)ceil_div(g.nb, ROWS), (unsigned)g.BH), dim3(256), smem, stream, g,
+                            qbar, kbarT, p, k_min, kv_cnt, kv_idx, probs, status);
 }
 
 template <int D>

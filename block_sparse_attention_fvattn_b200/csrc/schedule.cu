@@ -78,6 +78,8 @@ __global__ void __launch_bounds__(32 * kPairWarps) pair_lists_kernel(Geo g, cons
                                                                      int32_t *__restrict__ pair_list)
 {
     __shared__ uint32_t bm[kPairWarps][2][kMaxBlocks / 32];
+    pdl_release();
+    pdl_wait();  // the kept lists come from the routing kernels
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long pid = (long long)blockIdx.x * kPairWarps + warp;
     if (pid >= (long long)g.BH * g.npair) return;
@@ -129,9 +131,8 @@ cudaError_t launch_pair_lists(const Geo &g, const int32_t *kv_cnt, const int32_t
 {
     const long long pairs = (long long)g.BH * g.npair;
     if (pairs == 0) return cudaSuccess;
-    pair_lists_kernel<<<(unsigned)((pairs + kPairWarps - 1) / kPairWarps), 32 * kPairWarps, 0, stream>>>(
-        g, kv_cnt, kv_idx, pair_cnt, pair_list);
-    return cudaGetLastError();
+    return launch_dependent(pair_lists_kernel, dim3((unsigned)((pairs + kPairWarps - 1) / kPairWarps)),
+                            dim3(32 * kPairWarps), 0, stream, g, kv_cnt, kv_idx, pair_cnt, pair_list);
 }
 
 // Tiles of pair pp of head bh in paired mode: ceil(|union| / 2) steps of two
@@ -152,6 +153,8 @@ __global__ void __launch_bounds__(1024) sched_head_kernel(Geo g, const int32_t *
 {
     extern __shared__ unsigned long long keys[];
     __shared__ long long part[32];
+    pdl_release();
+    pdl_wait();  // kept lists or pair unions from the kernel before
     const int bh = blockIdx.x;
     const int hw = g.nbh * g.nbw;
     long long local = 0;
@@ -204,6 +207,8 @@ __global__ void __launch_bounds__(1024) sched_assign_kernel(Geo g, int C, const 
                                                             int64_t *__restrict__ cta_cost, int hpow2)
 {
     extern __shared__ unsigned long long sa_smem[];
+    pdl_release();
+    pdl_wait();  // unit costs from sched_head_kernel
     unsigned long long *hkeys = sa_smem;          // [hpow2]
     unsigned long long *ccost = sa_smem + hpow2;  // [C]
     for (int h = threadIdx.x; h < hpow2; h += blockDim.x) {
@@ -250,17 +255,16 @@ cudaError_t launch_schedule(const Geo &g, const int32_t *kv_cnt, const int32_t *
     const size_t smem_a = (size_t)npow2 * sizeof(unsigned long long);
     cudaError_t err = cudaFuncSetAttribute(sched_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a);
     if (err != cudaSuccess) return err;
-    sched_head_kernel<<<g.BH, 1024, smem_a, stream>>>(g, kv_cnt, kv_idx, dense, pair_cnt, unit_cost, head_sorted,
-                                                      head_cost, npow2);
-    err = cudaGetLastError();
+    err = launch_dependent(sched_head_kernel, dim3(g.BH), dim3(1024), smem_a, stream, g, kv_cnt, kv_idx, dense,
+                           pair_cnt, unit_cost, head_sorted, head_cost, npow2);
     if (err != cudaSuccess) return err;
     const int hpow2 = next_pow2(g.BH);
     const size_t smem_b = ((size_t)hpow2 + num_ctas) * sizeof(unsigned long long);
     err = cudaFuncSetAttribute(sched_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b);
     if (err != cudaSuccess) return err;
-    sched_assign_kernel<<<1, 1024, smem_b, stream>>>(g, num_ctas, unit_cost, head_sorted, head_cost, work,
-                                                     cta_range, cta_cost, hpow2);
-    return cudaGetLastError();
+    return launch_dependent(sched_assign_kernel, dim3(1), dim3(1024), smem_b, stream, g, num_ctas,
+                            (const int32_t *)unit_cost, (const int32_t *)head_sorted, (const int64_t *)head_cost,
+                            work, cta_range, cta_cost, hpow2);
 }
 
 }  // namespace fvattn
