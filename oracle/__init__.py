@@ -29,7 +29,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 
 
 class Geom(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "T", "Hg", "W", "D", "bt", "bh", "bw")]
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "T", "Hg", "W", "D", "bt", "bh", "bw", "fp16")]
 
 
 def compile_oracle(src: str = _SRC, out: str = _LIB) -> str:
@@ -53,11 +53,11 @@ def _ptr(a: Optional[np.ndarray]):
 
 
 def _as_u16(x) -> np.ndarray:
-    """bf16 tensor/array -> contiguous uint16 view of the raw bits (no rounding)."""
+    """bf16 or fp16 tensor/array -> contiguous uint16 view of the raw bits (no rounding)."""
     try:
         import torch
         if isinstance(x, torch.Tensor):
-            assert x.dtype == torch.bfloat16
+            assert x.dtype in (torch.bfloat16, torch.float16)
             return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
     except ImportError:  # pragma: no cover
         pass
@@ -78,15 +78,23 @@ class Oracle:
         L.oracle_num_blocks.restype = i32
         L.oracle_block_sizes.argtypes = [ctypes.POINTER(Geom), vp]
         L.oracle_pool.argtypes = [ctypes.POINTER(Geom), vp, vp]
+        L.oracle_widen.argtypes = [i32, vp, vp, ctypes.c_int64]
         L.oracle_route.argtypes = [ctypes.POINTER(Geom), vp, vp, f64, f64, i32, vp, vp, vp, vp, vp, vp]
         L.oracle_attn_rows.argtypes = [ctypes.POINTER(Geom), vp, vp, vp, f64, vp, vp,
                                        ctypes.c_int64, vp, vp, vp, vp, vp]
 
     @staticmethod
-    def geom(B, H, grid, block, D) -> Geom:
+    def geom(B, H, grid, block, D, fp16=False) -> Geom:
         T, Hg, W = grid
         bt, bh, bw = block
-        return Geom(B, H, T, Hg, W, D, bt, bh, bw)
+        return Geom(B, H, T, Hg, W, D, bt, bh, bw, 1 if fp16 else 0)
+
+    def widen(self, bits: np.ndarray, fp16: bool) -> np.ndarray:
+        """The oracle's exact decode of raw 16-bit elements to fp64."""
+        b = np.ascontiguousarray(bits, dtype=np.uint16)
+        out = np.zeros(b.size, dtype=np.float64)
+        self.lib.oracle_widen(ctypes.c_int32(1 if fp16 else 0), _ptr(b), _ptr(out), ctypes.c_int64(b.size))
+        return out
 
     def num_blocks(self, g: Geom) -> int:
         return int(self.lib.oracle_num_blocks(ctypes.byref(g)))

@@ -42,8 +42,10 @@
  *     [ai-feeds.com summary, "Key modules" 1 and the 4.41x result: attention
  *      is computed only over the kept blocks; zskr.cn guide, section 1.]
  *
- * All arithmetic is fp64 on bf16 inputs widened exactly. Loops are parallel
- * over independent (head, block) or (head, token) items only; the arithmetic
+ * All arithmetic is fp64 on the 16-bit inputs widened exactly: bfloat16
+ * (fp16 == 0) or IEEE 754 binary16 (fp16 == 1; the FastVideo VSA backend
+ * accepts both, zskr.cn guide, section 5). Loops are parallel over
+ * independent (head, block) or (head, token) items only; the arithmetic
  * inside each item runs in the plain order of its definition.
  */
 #include <math.h>
@@ -53,14 +55,40 @@
 
 typedef struct {
     int32_t B, H, T, Hg, W, D, bt, bh, bw;
+    int32_t fp16; /* element type of Q, K, V: 0 = bfloat16, 1 = IEEE binary16 */
 } oracle_geom;
 
+/* bfloat16: the upper half of an IEEE binary32. */
 static double bf16_to_f64(uint16_t h)
 {
     uint32_t u = ((uint32_t)h) << 16;
     float f;
     memcpy(&f, &u, sizeof f);
     return (double)f;
+}
+
+/* IEEE 754 binary16: sign, 5-bit exponent (bias 15), 10-bit fraction.
+ * Normal: (1024 + fraction) * 2^(exponent - 25); subnormal (exponent 0):
+ * fraction * 2^-24; exponent 31: infinity or NaN. */
+static double f16_to_f64(uint16_t h)
+{
+    const int sign = h >> 15, e = (h >> 10) & 0x1F, m = h & 0x3FF;
+    double v;
+    if (e == 0) v = ldexp((double)m, -24);
+    else if (e == 31) v = m ? NAN : INFINITY;
+    else v = ldexp((double)(1024 + m), e - 25);
+    return sign ? -v : v;
+}
+
+static double elem_to_f64(const oracle_geom *g, uint16_t h)
+{
+    return g->fp16 ? f16_to_f64(h) : bf16_to_f64(h);
+}
+
+/* Widen n raw 16-bit elements of the given type (for the checks of the decode). */
+void oracle_widen(int32_t fp16, const uint16_t *x, double *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = fp16 ? f16_to_f64(x[i]) : bf16_to_f64(x[i]);
 }
 
 static int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -124,7 +152,7 @@ void oracle_pool(const oracle_geom *g, const uint16_t *x, double *out)
                 for (int xx = x0; xx < x0 + xv; ++xx) {
                     const int64_t n = ((int64_t)t * g->Hg + y) * g->W + xx;
                     const uint16_t *row = x + (bh * N + n) * D;
-                    for (int d = 0; d < D; ++d) o[d] += bf16_to_f64(row[d]);
+                    for (int d = 0; d < D; ++d) o[d] += elem_to_f64(g, row[d]);
                 }
         const double cnt = (double)(tv * yv * xv);
         for (int d = 0; d < D; ++d) o[d] /= cnt;
@@ -264,7 +292,7 @@ void oracle_attn_rows(const oracle_geom *g, const uint16_t *q, const uint16_t *k
             const int64_t n = flat % N;
             const int i = token_block(g, n);
             const uint16_t *qr = q + (bh * N + n) * D;
-            for (int d = 0; d < D; ++d) qd[d] = bf16_to_f64(qr[d]);
+            for (int d = 0; d < D; ++d) qd[d] = elem_to_f64(g, qr[d]);
             int cnt = nb;
             const int32_t *lst = NULL;
             if (kv_cnt) {
@@ -283,7 +311,7 @@ void oracle_attn_rows(const oracle_geom *g, const uint16_t *q, const uint16_t *k
                             const int64_t m = ((int64_t)t * g->Hg + y) * g->W + x;
                             const uint16_t *kr = k + (bh * N + m) * D;
                             double dot = 0.0;
-                            for (int d = 0; d < D; ++d) dot += qd[d] * bf16_to_f64(kr[d]);
+                            for (int d = 0; d < D; ++d) dot += qd[d] * elem_to_f64(g, kr[d]);
                             logit[nk] = scale * dot;
                             key[nk] = m;
                             if (logit[nk] > mx) mx = logit[nk];
@@ -302,7 +330,7 @@ void oracle_attn_rows(const oracle_geom *g, const uint16_t *q, const uint16_t *k
                 ws += w;
                 const uint16_t *vr = v + (bh * N + key[e]) * D;
                 for (int d = 0; d < D; ++d) {
-                    const double vv = bf16_to_f64(vr[d]);
+                    const double vv = elem_to_f64(g, vr[d]);
                     acc[d] += w * vv;
                     if (lo) {
                         if (vv < lo[d]) lo[d] = vv;

@@ -270,8 +270,43 @@ def pin_nonfinite_repair(orc):
     assert (r["kv_cnt"][0, 0] < nb).any()
 
 
+# ---------------------------------------------------------------- input types
+def pin_element_decode(orc):
+    """The oracle widens every one of the 65536 bit patterns exactly like
+    numpy's IEEE binary16 and torch's bfloat16 conversions."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    for fp16 in (True, False):
+        got = orc.widen(bits, fp16)
+        if fp16:
+            ref = bits.view(np.float16).astype(np.float64)
+        else:
+            ref = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+        nan = np.isnan(ref)
+        assert np.array_equal(np.isnan(got), nan), fp16
+        assert np.array_equal(got[~nan], ref[~nan]), fp16
+
+
+def pin_fp16_inputs(orc):
+    """fp16 Q, K, V: pooling is a reshape-mean and p = 1 attention is torch's
+    scaled_dot_product_attention, both on the fp16 values widened to fp64."""
+    grid, block = (8, 16, 16), (4, 8, 8)
+    wl, q, k, v = _small(grid, block, H=2, D=32)
+    q16, k16, v16 = (t.float().to(torch.float16) for t in (q, k, v))
+    g = orc.geom(wl.B, wl.H, grid, block, wl.D, fp16=True)
+    qb = orc.pool(g, q16)
+    x = q16.double().numpy().reshape(1, wl.H, 2, 4, 2, 8, 2, 8, wl.D)
+    np.testing.assert_allclose(qb, x.mean(axis=(3, 5, 7)).reshape(1, wl.H, 8, wl.D), rtol=0, atol=1e-12)
+    kb = orc.pool(g, k16)
+    scale = 1.0 / math.sqrt(wl.D)
+    r = orc.route(g, qb, kb, scale, 1.0, 1)
+    rows = np.arange(wl.H * wl.N)
+    out, ws = orc.attn_rows(g, q16, k16, v16, scale, rows, r["kv_cnt"], r["kv_idx"])
+    ref = torch.nn.functional.scaled_dot_product_attention(q16.double(), k16.double(), v16.double())
+    np.testing.assert_allclose(out.reshape(1, wl.H, wl.N, wl.D), ref.numpy(), rtol=0, atol=1e-12)
+
+
 ALL_PINS = [
     pin_vsa_worked_example, pin_long_video_tokens, pin_pool_reshape_mean, pin_pool_ragged_bruteforce,
     pin_topp_bruteforce, pin_topk_reduction, pin_dense_reduction, pin_sparse_attention_masked_sdpa,
-    pin_invariants, pin_tie_order, pin_nonfinite_repair,
+    pin_invariants, pin_tie_order, pin_nonfinite_repair, pin_element_decode, pin_fp16_inputs,
 ]

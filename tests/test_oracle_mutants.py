@@ -37,6 +37,9 @@ MUTANTS = {
     "attn_ignores_lists": ("    if (kv_cnt) {\n                cnt", "    if (0) {\n                cnt"),
     "attn_missing_scale": ("logit[nk] = scale * dot;", "logit[nk] = dot;"),
     "attn_wrong_query_block": ("const int i = token_block(g, n);", "const int i = token_block(g, 0);"),
+    "f16_exponent_bias": ("else v = ldexp((double)(1024 + m), e - 25);", "else v = ldexp((double)(1024 + m), e - 24);"),
+    "f16_subnormal_scale": ("if (e == 0) v = ldexp((double)m, -24);", "if (e == 0) v = ldexp((double)m, -25);"),
+    "f16_inputs_read_as_bf16": ("return g->fp16 ? f16_to_f64(h) : bf16_to_f64(h);", "return bf16_to_f64(h);"),
 }
 
 
