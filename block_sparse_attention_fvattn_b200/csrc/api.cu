@@ -48,6 +48,7 @@ static fvattn_status resolve(const fvattn_problem *p, Geo *g)
     if ((long long)p->grid_t * p->grid_h * p->grid_w != (long long)p->N) return FVATTN_ERR_INVALID_ARG;
     if (isnan(p->softmax_scale) || isinf(p->softmax_scale)) return FVATTN_ERR_INVALID_ARG;
     if (p->D != 64 && p->D != 128) return FVATTN_ERR_UNSUPPORTED;
+    if (p->dtype != FVATTN_DTYPE_BF16 && p->dtype != FVATTN_DTYPE_F16) return FVATTN_ERR_UNSUPPORTED;
     const long long bp = (long long)p->blk_t * p->blk_h * p->blk_w;
     if (!(bp == 256 && p->blk_t % 2 == 0) && bp != 64) return FVATTN_ERR_UNSUPPORTED;
     if (p->blk_w > 256 || p->blk_h > 256 || p->blk_t > 256) return FVATTN_ERR_UNSUPPORTED;
@@ -58,6 +59,7 @@ static fvattn_status resolve(const fvattn_problem *p, Geo *g)
     G.H = p->H;
     G.N = p->N;
     G.D = p->D;
+    G.f16 = p->dtype == FVATTN_DTYPE_F16 ? 1 : 0;
     G.T = p->grid_t;
     G.Hg = p->grid_h;
     G.W = p->grid_w;

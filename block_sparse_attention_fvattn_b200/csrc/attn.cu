@@ -280,13 +280,13 @@ __device__ __forceinline__ void exp2_poly_x2(uint64_t a, float &p0, float &p1)
     p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
-template <int D, int BKV, bool PAIRED>
+template <int D, int BKV, bool PAIRED, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, Geo g, const int32_t *__restrict__ kv_cnt,
                 const int32_t *__restrict__ kv_idx, const int32_t *__restrict__ pair_cnt,
                 const int32_t *__restrict__ pair_list, const int32_t *__restrict__ work,
-                const int32_t *__restrict__ cta_range, int dense, __nv_bfloat16 *__restrict__ out,
+                const int32_t *__restrict__ cta_range, int dense, uint16_t *__restrict__ out,
                 int64_t *__restrict__ cta_ns, uint32_t *__restrict__ status)
 {
     static_assert(!PAIRED || BKV == 128, "paired mode runs 128-token key/value tiles");
@@ -494,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ================= QK issuer =================
         if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16(128, BKV, false);
+            constexpr uint32_t idesc_qk = idesc_16(128, BKV, false, F16);
             // descriptors of the first slab of each region; every other operand
             // is a fixed byte offset from it (added to the start-address field)
             const uint64_t q_desc = sdesc_sw128(sbase + L::kQ, 16, 1024);
@@ -580,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 2) {
         // ================= PV issuer =================
         if (lane == 0) {
-            constexpr uint32_t idesc_pv = idesc_bf16(128, D, true);
+            constexpr uint32_t idesc_pv = idesc_16(128, D, true, F16);
             const uint64_t v_desc = sdesc_sw128(sbase + L::kV, L::kKVSlab, 1024);
             int vc = 0;
             uint32_t ph_p = 0, ph_oe = 0, o_pend = 0;
@@ -755,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     p1 = ex2_approx(a1);
                 }
                 s4[q2 & 3] = f2_add(s4[q2 & 3], f2_pack(p0, p1));
-                pk[q2] = pack_bf16x2(p0, p1);
+                pk[q2] = pack16x2<F16>(p0, p1);
             }
             float sum;
             {
@@ -795,7 +795,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++of;
             tc_fence_after();
             const float inv = 1.0f / l;
-            __nv_bfloat16 *orow =
+            uint16_t *orow =
                 out + ((size_t)ubh * g.N + ((size_t)qt * g.Hg + qy) * g.W + qx) * (size_t)D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
@@ -807,10 +807,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
                         uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(o[q4 * 8 + 0]) * inv, __uint_as_float(o[q4 * 8 + 1]) * inv);
-                        w.y = pack_bf16x2(__uint_as_float(o[q4 * 8 + 2]) * inv, __uint_as_float(o[q4 * 8 + 3]) * inv);
-                        w.z = pack_bf16x2(__uint_as_float(o[q4 * 8 + 4]) * inv, __uint_as_float(o[q4 * 8 + 5]) * inv);
-                        w.w = pack_bf16x2(__uint_as_float(o[q4 * 8 + 6]) * inv, __uint_as_float(o[q4 * 8 + 7]) * inv);
+                        w.x = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 0]) * inv, __uint_as_float(o[q4 * 8 + 1]) * inv);
+                        w.y = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 2]) * inv, __uint_as_float(o[q4 * 8 + 3]) * inv);
+                        w.z = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 4]) * inv, __uint_as_float(o[q4 * 8 + 5]) * inv);
+                        w.w = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 6]) * inv, __uint_as_float(o[q4 * 8 + 7]) * inv);
                         dst[q4] = w;
                     }
                 }
@@ -974,20 +974,21 @@ static bool make_map(CUtensorMap *map, const Geo &g, const void *ptr)
                                    (cuuint64_t)g.Hg * g.W * g.D * es, (cuuint64_t)g.N * g.D * es};
     const cuuint32_t box[5] = {64u, (cuuint32_t)g.bw, (cuuint32_t)g.bh, (cuuint32_t)g.subt, 1u};
     const cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(ptr), dims, strides, box, estr,
+    CUresult r = enc(map, g.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
+                     const_cast<void *>(ptr), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
-template <int D, int BKV, bool PAIRED>
-static cudaError_t launch_attn_t(const Geo &g, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+template <int D, int BKV, bool PAIRED, bool F16>
+static cudaError_t launch_attn_f(const Geo &g, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                                  const int32_t *kv_cnt, const int32_t *kv_idx, const int32_t *pair_cnt,
                                  const int32_t *pair_list, const int32_t *work, const int32_t *cta_range, int grid,
                                  int dense, void *out, int64_t *cta_ns, uint32_t *status, cudaStream_t stream)
 {
     using L = AttnLayout<D, BKV, PAIRED>;
-    auto kern = attn_kernel<D, BKV, PAIRED>;
+    auto kern = attn_kernel<D, BKV, PAIRED, F16>;
     cudaFuncAttributes fa;
     cudaError_t err = cudaFuncGetAttributes(&fa, kern);
     if (err != cudaSuccess) return err;
@@ -998,7 +999,20 @@ static cudaError_t launch_attn_t(const Geo &g, const CUtensorMap &mq, const CUte
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (err != cudaSuccess) return err;
     return launch_dependent(kern, dim3(grid), dim3(kThreads), L::kAlloc, stream, mq, mk, mv, g, kv_cnt, kv_idx,
-                            pair_cnt, pair_list, work, cta_range, dense, (__nv_bfloat16 *)out, cta_ns, status);
+                            pair_cnt, pair_list, work, cta_range, dense, (uint16_t *)out, cta_ns, status);
+}
+
+template <int D, int BKV, bool PAIRED>
+static cudaError_t launch_attn_t(const Geo &g, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                                 const int32_t *kv_cnt, const int32_t *kv_idx, const int32_t *pair_cnt,
+                                 const int32_t *pair_list, const int32_t *work, const int32_t *cta_range, int grid,
+                                 int dense, void *out, int64_t *cta_ns, uint32_t *status, cudaStream_t stream)
+{
+    if (g.f16)
+        return launch_attn_f<D, BKV, PAIRED, true>(g, mq, mk, mv, kv_cnt, kv_idx, pair_cnt, pair_list, work,
+                                                   cta_range, grid, dense, out, cta_ns, status, stream);
+    return launch_attn_f<D, BKV, PAIRED, false>(g, mq, mk, mv, kv_cnt, kv_idx, pair_cnt, pair_list, work, cta_range,
+                                                grid, dense, out, cta_ns, status, stream);
 }
 
 cudaError_t launch_attn(const Geo &g, const void *q, const void *k, const void *v, const int32_t *kv_cnt,

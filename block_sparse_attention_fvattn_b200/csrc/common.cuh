@@ -8,6 +8,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -45,6 +46,7 @@ struct Geo {
     int subt;              // frames per 128-/64-row sub-tile (bt/2 for 256-token blocks, bt for 64)
     int nsub;              // sub-tiles per block along t (2 or 1)
     int rows;              // rows per sub-tile (128 or 64)
+    int f16;               // Q, K, V, O are IEEE fp16 (else bf16)
     int paired;            // 64-token blocks: two query blocks share one 128-row tile
     int npair;             // pairs of query blocks (2p, 2p+1) per head: ceil(nb/2) when paired
     int upb;               // attention work units per (b, h): nb, or ceil(nb/4) when paired
@@ -302,10 +304,12 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
 
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, A K-major,
 // B K-major (QK^T) or MN-major (PV), N>>3 in bits 17-22, M>>4 in bits 24-28.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
+// Instruction descriptor of tcgen05.mma kind::f16 with fp32 accumulation:
+// A and B both bf16 (format 1) or both fp16 (format 0).
+__host__ __device__ constexpr uint32_t idesc_16(int M, int N, bool b_mn_major, bool f16)
 {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
-           ((uint32_t)(M >> 4) << 24);
+    return (1u << 4) | ((f16 ? 0u : 1u) << 7) | ((f16 ? 0u : 1u) << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 // sm_100 three-input max and packed fp32x2 arithmetic
@@ -349,6 +353,31 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
+{
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+// Two floats rounded to the 16-bit element type and packed (lo in the low half).
+template <bool F16>
+__device__ __forceinline__ uint32_t pack16x2(float lo, float hi)
+{
+    if constexpr (F16) return pack_f16x2(lo, hi);
+    else return pack_bf16x2(lo, hi);
+}
+// The two 16-bit elements of a word, widened (exactly) to fp32.
+template <bool F16>
+__device__ __forceinline__ void unpack16x2(uint32_t w, float &lo, float &hi)
+{
+    if constexpr (F16) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w));
+        lo = f.x;
+        hi = f.y;
+    } else {
+        lo = __uint_as_float(w << 16);
+        hi = __uint_as_float(w & 0xFFFF0000u);
+    }
 }
 
 // Launch `kern` as a programmatic dependent of the previous kernel on `stream`.

@@ -49,9 +49,9 @@ __host__ __device__ inline PoolPlan pool_plan(int nbw, int bw, int D)
     return pl;
 }
 
-template <int D, int NS>
-__global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geo g, int nxs, const __nv_bfloat16 *__restrict__ q,
-                                                            const __nv_bfloat16 *__restrict__ k,
+template <int D, int NS, bool F16>
+__global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geo g, int nxs, const uint16_t *__restrict__ q,
+                                                            const uint16_t *__restrict__ k,
                                                             float *__restrict__ qbar, float *__restrict__ kbarT)
 {
     constexpr int LPT = D / 8;  // 16-byte chunks per token
@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geo g, int nxs, cons
     const int npos = (x1 - x0) * LPT;
     const int tid = threadIdx.x;
 
-    const __nv_bfloat16 *src = which ? k : q;
+    const uint16_t *src = which ? k : q;
     const uint4 *run = reinterpret_cast<const uint4 *>(src + (size_t)bh * g.N * D) +
                        (((size_t)t0 * g.Hg + y0) * g.W + x0) * LPT;
     const size_t run_step = (size_t)g.W * LPT;                            // next y
@@ -121,8 +121,11 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geo g, int nxs, cons
                         const uint32_t w[4] = {v[b][s].x, v[b][s].y, v[b][s].z, v[b][s].w};
 #pragma unroll
                         for (int c = 0; c < 4; ++c)
-                            acc[s][c] = f2_add(acc[s][c], f2_pack(__uint_as_float(w[c] << 16),
-                                                                  __uint_as_float(w[c] & 0xFFFF0000u)));
+                        {
+                            float lo, hi;
+                            unpack16x2<F16>(w[c], lo, hi);
+                            acc[s][c] = f2_add(acc[s][c], f2_pack(lo, hi));
+                        }
                     }
                 }
             }
@@ -670,18 +673,26 @@ __global__ void __launch_bounds__(256, kSelMinBlocksFor<EPL>) score_select_kerne
 }
 
 // ---------------------------------------------------------------------------
+template <int D, int NS, bool F16>
+static cudaError_t launch_pool_f(const Geo &g, int nxs, const void *q, const void *k, float *qbar, float *kbarT,
+                                 cudaStream_t stream)
+{
+    const size_t smem = (size_t)kPoolThreads * NS * 8 * sizeof(float);
+    auto kern = pool_kernel<D, NS, F16>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    const long long blocks = 2ll * g.BH * g.nbt * g.nbh * nxs;
+    kern<<<(unsigned)blocks, kPoolThreads, smem, stream>>>(g, nxs, (const uint16_t *)q, (const uint16_t *)k, qbar,
+                                                          kbarT);
+    return cudaGetLastError();
+}
+
 template <int D, int NS>
 static cudaError_t launch_pool_t(const Geo &g, int nxs, const void *q, const void *k, float *qbar, float *kbarT,
                                  cudaStream_t stream)
 {
-    const size_t smem = (size_t)kPoolThreads * NS * 8 * sizeof(float);
-    auto kern = pool_kernel<D, NS>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    const long long blocks = 2ll * g.BH * g.nbt * g.nbh * nxs;
-    kern<<<(unsigned)blocks, kPoolThreads, smem, stream>>>(g, nxs, (const __nv_bfloat16 *)q,
-                                                          (const __nv_bfloat16 *)k, qbar, kbarT);
-    return cudaGetLastError();
+    if (g.f16) return launch_pool_f<D, NS, true>(g, nxs, q, k, qbar, kbarT, stream);
+    return launch_pool_f<D, NS, false>(g, nxs, q, k, qbar, kbarT, stream);
 }
 
 template <int D>

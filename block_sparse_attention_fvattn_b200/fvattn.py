@@ -28,9 +28,14 @@ class FVAttnError(RuntimeError):
         super().__init__(f"{where}: {status_string(status)} (status {status})")
 
 
+DTYPE_BF16, DTYPE_F16 = 0, 1
+_DTYPES = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_F16}
+
+
 class Problem(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "N", "D", "grid_t", "grid_h", "grid_w",
-                                              "blk_t", "blk_h", "blk_w")] + [("softmax_scale", ctypes.c_float)]
+                                              "blk_t", "blk_h", "blk_w")] + [("softmax_scale", ctypes.c_float),
+                                                                             ("dtype", ctypes.c_int32)]
 
 
 def _load():
@@ -77,6 +82,7 @@ class Geometry:
     grid: Tuple[int, int, int]
     block: Tuple[int, int, int]
     softmax_scale: float = 0.0   # <= 0 selects 1/sqrt(D)
+    dtype: torch.dtype = torch.bfloat16  # element type of Q, K, V, O: bfloat16 or float16
 
     @property
     def N(self) -> int:
@@ -85,7 +91,10 @@ class Geometry:
     def problem(self) -> Problem:
         T, Hg, W = self.grid
         bt, bh, bw = self.block
-        return Problem(self.B, self.H, self.N, self.D, T, Hg, W, bt, bh, bw, float(self.softmax_scale))
+        if self.dtype not in _DTYPES:
+            raise ValueError(f"unsupported element type {self.dtype}; use torch.bfloat16 or torch.float16")
+        return Problem(self.B, self.H, self.N, self.D, T, Hg, W, bt, bh, bw, float(self.softmax_scale),
+                       _DTYPES[self.dtype])
 
     @property
     def scale(self) -> float:
@@ -137,7 +146,7 @@ def route(geo: Geometry, q: torch.Tensor, k: torch.Tensor, p: float, k_min: int,
           kv_cnt: torch.Tensor, kv_idx: torch.Tensor, ws: torch.Tensor,
           block_probs: Optional[torch.Tensor] = None, stream=None):
     prob = geo.problem()
-    st = _lib.fvattn_route(ctypes.byref(prob), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+    st = _lib.fvattn_route(ctypes.byref(prob), _ptr(q, geo.dtype, "q"), _ptr(k, geo.dtype, "k"),
                            float(p), int(k_min), _ptr(kv_cnt, torch.int32, "kv_cnt"),
                            _ptr(kv_idx, torch.int32, "kv_idx"), _ptr(block_probs, torch.float32, "block_probs"),
                            _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
@@ -152,7 +161,7 @@ def route_noalloc(geo: Geometry, q: torch.Tensor, k: torch.Tensor, p: float, k_m
     Calls that may overlap on the GPU race on that array; order them on one
     stream, and make the first call on a device before any stream capture."""
     prob = geo.problem()
-    st = _lib.fvattn_route_noalloc(ctypes.byref(prob), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+    st = _lib.fvattn_route_noalloc(ctypes.byref(prob), _ptr(q, geo.dtype, "q"), _ptr(k, geo.dtype, "k"),
                                    float(p), int(k_min), _ptr(kv_cnt, torch.int32, "kv_cnt"),
                                    _ptr(kv_idx, torch.int32, "kv_idx"),
                                    _ptr(block_probs, torch.float32, "block_probs"), _stream(stream))
@@ -174,11 +183,11 @@ def schedule(geo: Geometry, kv_cnt: Optional[torch.Tensor], kv_idx: Optional[tor
 def sparse_attn(geo: Geometry, q, k, v, kv_cnt, kv_idx, work, cta_range, num_ctas: int, dense: bool,
                 out: torch.Tensor, ws: torch.Tensor, cta_ns: Optional[torch.Tensor] = None, stream=None):
     prob = geo.problem()
-    st = _lib.fvattn_sparse_attn(ctypes.byref(prob), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
-                                 _ptr(v, torch.bfloat16, "v"), _ptr(kv_cnt, torch.int32, "kv_cnt"),
+    st = _lib.fvattn_sparse_attn(ctypes.byref(prob), _ptr(q, geo.dtype, "q"), _ptr(k, geo.dtype, "k"),
+                                 _ptr(v, geo.dtype, "v"), _ptr(kv_cnt, torch.int32, "kv_cnt"),
                                  _ptr(kv_idx, torch.int32, "kv_idx"), _ptr(work, torch.int32, "work"),
                                  _ptr(cta_range, torch.int32, "cta_range"), int(num_ctas), int(bool(dense)),
-                                 _ptr(out, torch.bfloat16, "out"), _ptr(cta_ns, torch.int64, "cta_ns"),
+                                 _ptr(out, geo.dtype, "out"), _ptr(cta_ns, torch.int64, "cta_ns"),
                                  _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
     _check(st, "fvattn_sparse_attn")
 

@@ -18,8 +18,9 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- * Tensors.  Q, K, V and O are bf16, contiguous, [B, H, N, D] (row-major, D
- *   innermost). Token n of a head sits at latent position (t, y, x) with
+ * Tensors.  Q, K, V and O are bf16 or fp16 (fvattn_problem.dtype), contiguous,
+ *   [B, H, N, D] (row-major, D innermost). Attention runs the products on the
+ *   tensor cores in that type with fp32 accumulation; P is rounded to it too. Token n of a head sits at latent position (t, y, x) with
  *   n = (t * grid_h + y) * grid_w + x (raster order, T slowest), as in the
  *   FastVideo VSA backend's (T, H, W) post-patch latent grid (zskr.cn guide,
  *   section 1). Q and KV have the same length (non-causal self-attention,
@@ -81,11 +82,17 @@ typedef enum fvattn_status {
 #define FVATTN_FLAG_NONFINITE 0x1u
 #define FVATTN_FLAG_TIMEOUT 0x2u
 
+/* Element type of Q, K, V and O (the FastVideo VSA backend accepts both,
+ * zskr.cn guide, section 5). */
+#define FVATTN_DTYPE_BF16 0
+#define FVATTN_DTYPE_F16 1
+
 typedef struct fvattn_problem {
     int32_t B, H, N, D;               /* batch, heads, tokens (= T*Hg*W), head dim */
     int32_t grid_t, grid_h, grid_w;   /* latent grid (T, H, W) */
     int32_t blk_t, blk_h, blk_w;      /* block shape */
     float softmax_scale;              /* <= 0 selects 1/sqrt(D); used for routing and attention */
+    int32_t dtype;                    /* FVATTN_DTYPE_BF16 or FVATTN_DTYPE_F16; other values: UNSUPPORTED */
 } fvattn_problem;
 
 /* nb = ceil(T/bt)*ceil(H/bh)*ceil(W/bw), or -1 if the problem is invalid. */

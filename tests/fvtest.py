@@ -28,13 +28,16 @@ TOPP_WINDOW = 1e-5
 TIE_FACTOR = 4e-5
 
 
-def geometry(wl):
+def geometry(wl, dtype=torch.bfloat16):
     from block_sparse_attention_fvattn_b200 import fvattn as fa
-    return fa.Geometry(wl.B, wl.H, wl.D, wl.grid, wl.block)
+    return fa.Geometry(wl.B, wl.H, wl.D, wl.grid, wl.block, dtype=dtype)
 
 
-def make_on_gpu(wl, seed=None):
+def make_on_gpu(wl, seed=None, dtype=torch.bfloat16):
+    """The seeded bf16 inputs; for fp16 they are converted (through fp32)."""
     q, k, v = gen.make_inputs(wl, "cuda", seed=seed)
+    if dtype != torch.bfloat16:
+        q, k, v = (t.float().to(dtype) for t in (q, k, v))
     torch.cuda.synchronize()
     return q, k, v
 

@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "fvattn.h")
@@ -63,6 +64,17 @@ def test_problem_validation(fa, geo_args, expect):
                               ctypes.c_void_p(0x1000), ctypes.c_void_p(0x1000), None, ctypes.c_void_p(0x1000),
                               1 << 30, None)
     assert st == getattr(fa, expect)
+
+
+def test_element_type(fa):
+    # bf16 and fp16 are accepted; any other element type code is UNSUPPORTED
+    for code, ok in ((fa.DTYPE_BF16, True), (fa.DTYPE_F16, True), (2, False), (-1, False)):
+        p = fa.Geometry(1, 1, 128, (8, 16, 16), (4, 8, 8)).problem()
+        p.dtype = code
+        assert (fa._lib.fvattn_num_blocks(ctypes.byref(p)) == 8) == ok, code
+    assert fa.Geometry(1, 1, 128, (8, 16, 16), (4, 8, 8), dtype=torch.float16).problem().dtype == fa.DTYPE_F16
+    with pytest.raises(ValueError):
+        fa.Geometry(1, 1, 128, (8, 16, 16), (4, 8, 8), dtype=torch.float32).problem()
 
 
 def test_grid_product_must_equal_n(fa):

@@ -35,7 +35,7 @@ FULL = [gen.WORKLOADS[n] for n in gen.WORKLOAD_ORDER]
 
 
 def _oracle_route(orc, wl, q, k):
-    g = orc.geom(wl.B, wl.H, wl.grid, wl.block, wl.D)
+    g = orc.geom(wl.B, wl.H, wl.grid, wl.block, wl.D, fp16=q.dtype == torch.float16)
     qb, kb = orc.pool(g, q), orc.pool(g, k)
     r = orc.route(g, qb, kb, 1.0 / math.sqrt(wl.D), wl.p, wl.k_min)
     return g, qb, kb, r
@@ -99,12 +99,12 @@ def _expected_work(cost, C):
     return lists
 
 
-def _run(wl, full_rows):
+def _run(wl, full_rows, dtype=torch.bfloat16):
     import oracle
     from block_sparse_attention_fvattn_b200 import fvattn as fa
     orc = oracle.get()
-    q, k, v = fvtest.make_on_gpu(wl)
-    geo = fvtest.geometry(wl)
+    q, k, v = fvtest.make_on_gpu(wl, dtype=dtype)
+    geo = fvtest.geometry(wl, dtype)
     eng = fa.FVAttn(geo, wl.p, wl.k_min, with_probs=True)
     eng.route(q, k)
     eng.schedule()
@@ -164,6 +164,12 @@ def _run(wl, full_rows):
 @pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
 def test_small_every_row(wl):
     _run(wl, full_rows=True)
+
+
+@pytest.mark.parametrize("name", ["ragged_256tok", "blk64", "blk64_ragged_d64"])
+def test_small_fp16_every_row(name):
+    # fp16 Q, K, V: the same path with fp16 TMA tiles, fp16 MMAs and fp16 P and O
+    _run([w for w in SMALL if w.name == name][0], full_rows=True, dtype=torch.float16)
 
 
 @pytest.mark.parametrize("wl", FULL, ids=lambda w: w.name)
