@@ -292,8 +292,11 @@ def run_gpu(args, wl, world, rank, local):
     pk, pk_src = peaks()
     seed = wl.seed + 1000 * rank
     q, k, v = gen.make_inputs(wl, dev, seed=seed)
+    edtype = torch.float16 if args.dtype == "f16" else torch.bfloat16
+    if edtype != torch.bfloat16:
+        q, k, v = (t.float().to(edtype) for t in (q, k, v))
     out = torch.empty_like(q)
-    geo = fa.Geometry(wl.B, wl.H, wl.D, wl.grid, wl.block)
+    geo = fa.Geometry(wl.B, wl.H, wl.D, wl.grid, wl.block, dtype=edtype)
     eng = fa.FVAttn(geo, wl.p, wl.k_min, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -415,7 +418,7 @@ def run_gpu(args, wl, world, rank, local):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
         "config": {"workload": workload_desc(wl), "parallelism": f"replicas x{world} (heads shard, no exchange)",
                    "l2": f"inputs {3 * q.numel() * 2 / 1e6:.0f} MB per step > L2, no flush",
                    "seed": seed, "num_ctas": eng.num_ctas},
@@ -432,7 +435,8 @@ def run_gpu(args, wl, world, rank, local):
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": attn_tflops / peak_tf, "traffic": traffic,
                      "kernel": f"attn_kernel<{wl.D},128,{'paired' if paired else 'unpaired'}> (fvattn_sparse_attn)",
-                     "peak_source": f"{pk_src} bf16 burst" + ("" if pk_src == "measured" else " (fallback)")},
+                     "peak_source": f"{pk_src} bf16 burst" + ("" if pk_src == "measured" else " (fallback)")
+                     + (" x 1 (fp16 has the bf16 dense rate)" if args.dtype == "f16" else "")},
         "route_roofline": {"bound": "hbm", "achieved": route_bytes / (route_avg * 1e-3) / 1e9,
                            "peak": pk["hbm_gbs"], "unit": "GB/s",
                            "frac": route_bytes / (route_avg * 1e-3) / 1e9 / pk["hbm_gbs"]},
@@ -456,6 +460,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle attention work")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--dtype", default="bf16", choices=["bf16", "f16"], help="element type of Q, K, V and O")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
