@@ -257,3 +257,72 @@ class FVAttn:
 
     def status(self, stream=None) -> int:
         return read_device_status(self.ws, stream)
+
+
+class HostPipeline:
+    """The whole path on host-resident (pinned) Q, K, V, O, with the
+    host<->device copies overlapped with the compute.
+
+    Heads are independent all along the path, so the B*H heads are split into
+    `groups` contiguous ranges, each run as its own problem (B=1, H=its heads)
+    through the same three library calls. Group c+1 is copied in on one stream
+    while group c computes on the caller's stream and group c-1 is copied out
+    on a third, so a call takes about the host->device copy time plus one
+    group's compute and copy-out. The result is the same as FVAttn on the
+    whole problem (every head is routed, scheduled and attended alone).
+    """
+
+    def __init__(self, geo: Geometry, p: float, k_min: int, groups: int = 4, device="cuda", num_ctas: int = 0):
+        BH = geo.B * geo.H
+        groups = max(1, min(int(groups), BH))
+        self.geo, self.dev = geo, torch.device(device)
+        self.ranges = [(BH * c // groups, BH * (c + 1) // groups) for c in range(groups)]
+        self.engines = [FVAttn(Geometry(1, h1 - h0, geo.D, geo.grid, geo.block, geo.softmax_scale, geo.dtype),
+                               p, k_min, device=device, num_ctas=num_ctas) for h0, h1 in self.ranges]
+        shape = (BH, geo.N, geo.D)
+        self.dq, self.dk, self.dv, self.dout = (torch.empty(shape, dtype=geo.dtype, device=self.dev) for _ in range(4))
+        self.s_in = torch.cuda.Stream(device=self.dev)
+        self.s_out = torch.cuda.Stream(device=self.dev)
+
+    def __call__(self, hq: torch.Tensor, hk: torch.Tensor, hv: torch.Tensor, hout: torch.Tensor):
+        """hq, hk, hv, hout: pinned host tensors [B, H, N, D] of the problem's dtype.
+        Enqueued on the current stream; returns without waiting, like the
+        library calls (synchronise before reading hout)."""
+        for t, name in ((hq, "q"), (hk, "k"), (hv, "v"), (hout, "out")):
+            if t.is_cuda or not t.is_pinned():
+                raise ValueError(f"{name} must be a pinned host tensor")
+            if t.dtype != self.geo.dtype or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous {self.geo.dtype} tensor")
+            if tuple(t.shape) != (self.geo.B, self.geo.H, self.geo.N, self.geo.D):
+                raise ValueError(f"{name} has shape {tuple(t.shape)}")
+        BH = self.geo.B * self.geo.H
+        views = [t.view(BH, self.geo.N, self.geo.D) for t in (hq, hk, hv, hout)]
+        compute = torch.cuda.current_stream(self.dev)
+        self.s_in.wait_stream(compute)   # the device buffers are free once earlier work is done
+        self.s_out.wait_stream(compute)
+        copied, done = [], []
+        for h0, h1 in self.ranges:
+            with torch.cuda.stream(self.s_in):
+                for dst, src in zip((self.dq, self.dk, self.dv), views[:3]):
+                    dst[h0:h1].copy_(src[h0:h1], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(self.s_in)
+                copied.append(ev)
+        for (h0, h1), eng, ev in zip(self.ranges, self.engines, copied):
+            compute.wait_event(ev)
+            eng(self.dq[h0:h1], self.dk[h0:h1], self.dv[h0:h1], out=self.dout[h0:h1])
+            d = torch.cuda.Event()
+            d.record(compute)
+            done.append(d)
+        for (h0, h1), d in zip(self.ranges, done):
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(d)
+                views[3][h0:h1].copy_(self.dout[h0:h1], non_blocking=True)
+        compute.wait_stream(self.s_out)
+        return hout
+
+    def status(self) -> int:
+        flags = 0
+        for eng in self.engines:
+            flags |= eng.status()
+        return flags
