@@ -378,6 +378,23 @@ def run_gpu(args, wl, world, rank, local):
     imb_meas = float(cta_ns[busy].max() / cta_ns[busy].mean()) if busy.any() else 1.0
     status = eng.status()
 
+    # ---- the same step replayed as one CUDA graph (no per-kernel events inside)
+    graph_ms = None
+    if not args.no_graph:
+        graph = eng.capture(q, k, v, out)
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        graph_ms = max_over_ranks(a.elapsed_time(b), world) / args.steps
+        del graph
+
     # ---- end to end through the public API with host buffers: HostPipeline
     # copies Q, K, V in and O out per group of heads, overlapped with the
     # compute of the neighbouring groups
@@ -440,6 +457,7 @@ def run_gpu(args, wl, world, rank, local):
                            "frac": route_bytes / (route_avg * 1e-3) / 1e9 / pk["hbm_gbs"]},
         "clocks": clk,
         # per step: pool + select (route), [pair lists +] two scheduler kernels, attention
+        "graph_ms_per_step": graph_ms,
         "gpu_launches": (6 if paired else 5) * args.steps,
         "e2e": e2e,
         "cpu_baseline": cpu,
@@ -460,6 +478,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "f16"], help="element type of Q, K, V and O")
     ap.add_argument("--e2e-groups", type=int, default=8, help="head groups of the host-buffer pipeline")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -258,6 +258,23 @@ class FVAttn:
     def status(self, stream=None) -> int:
         return read_device_status(self.ws, stream)
 
+    def capture(self, q, k, v, out) -> torch.cuda.CUDAGraph:
+        """Record route -> schedule -> attention on fixed q, k, v, out as one CUDA
+        graph; `graph.replay()` then runs the whole step with one launch call.
+        The kernels' programmatic launch dependencies become graph edges, and
+        the counters they share through the workspace reset themselves, so
+        the graph can be replayed any number of times."""
+        self(q, k, v, out)  # first use outside the capture: attributes and tensor-map encoder
+        torch.cuda.synchronize(q.device)
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device=q.device)
+        side.wait_stream(torch.cuda.current_stream(q.device))
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side):
+                self(q, k, v, out)
+        torch.cuda.current_stream(q.device).wait_stream(side)
+        return graph
+
 
 class HostPipeline:
     """The whole path on host-resident (pinned) Q, K, V, O, with the

@@ -155,6 +155,22 @@ def test_host_pipeline_matches_device_path(groups):
     assert torch.equal(hout, ref.cpu())
 
 
+@pytest.mark.parametrize("block", [(4, 8, 8), (4, 4, 4)])
+def test_cuda_graph_replay_matches_eager(block):
+    wl = gen.custom("graph", 1, 3, 128, (9, 20, 28), block, 0.9, 4, sigma=2.0, a_range=(0.5, 4.0), seed=40)
+    q, k, v = fvtest.make_on_gpu(wl)
+    eng = _engine(wl)
+    ref = eng(q, k, v).clone()
+    out = torch.zeros_like(q)
+    graph = eng.capture(q, k, v, out)
+    out.zero_()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert eng.status() == 0
+    assert torch.equal(out, ref)
+
+
 def test_repeatable():
     wl = gen.WORKLOADS["wan5b"]
     q, k, v = fvtest.make_on_gpu(wl)
