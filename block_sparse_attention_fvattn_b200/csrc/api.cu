@@ -27,8 +27,11 @@ WsLayout ws_layout(const Geo &g)
         off = align256(off + bytes);
         return o;
     };
-    L.qbar = take((size_t)g.BH * g.nb * g.D * sizeof(float));
-    L.kbarT = take((size_t)g.BH * g.D * g.nbp * sizeof(float));
+    // with tc_scores both hold two planes (the TF32 head and rest of each mean)
+    const size_t planes = g.tc_scores ? 2 : 1;
+    L.qbar = take(planes * g.BH * g.nb * g.D * sizeof(float));
+    L.kbarT = take(planes * g.BH * g.D * g.nbp * sizeof(float));
+    L.scores = take(g.tc_scores ? (size_t)g.BH * g.nb * g.nbp * sizeof(float) : 0);
     L.unit_cost = take((size_t)g.BH * g.nb * sizeof(int32_t));
     L.head_sorted = take((size_t)g.BH * g.nb * sizeof(int32_t));
     L.head_cost = take((size_t)g.BH * sizeof(int64_t));
@@ -85,6 +88,7 @@ static fvattn_status resolve(const fvattn_problem *p, Geo *g)
         G.nsub = 1;
         G.rows = 64;
     }
+    G.tc_scores = G.nb >= kTcScoresMinBlocks ? 1 : 0;
     G.paired = G.rows == 64;
     G.npair = G.paired ? ceil_div(G.nb, 2) : 0;
     G.upb = G.paired ? ceil_div(G.nb, 4) : G.nb;
@@ -164,8 +168,13 @@ fvattn_status fvattn_route(const fvattn_problem *prob, const void *q, const void
     float *kbarT = reinterpret_cast<float *>(w + L.kbarT);
     uint32_t *status = reinterpret_cast<uint32_t *>(w);
     cudaStream_t s = (cudaStream_t)stream;
+    float *scores = g.tc_scores ? reinterpret_cast<float *>(w + L.scores) : nullptr;
     if (launch_pool(g, q, k, qbar, kbarT, s) != cudaSuccess) return FVATTN_ERR_CUDA;
-    if (launch_score_select(g, qbar, kbarT, p, k_min, kv_cnt, kv_idx, block_probs, status, s) != cudaSuccess)
+    if (scores && launch_score_gemm(g, qbar, qbar + (size_t)g.BH * g.nb * g.D, kbarT,
+                                    kbarT + (size_t)g.BH * g.nbp * g.D, scores, status, s) != cudaSuccess)
+        return FVATTN_ERR_CUDA;
+    if (launch_score_select(g, qbar, kbarT, scores, p, k_min, kv_cnt, kv_idx, block_probs, status, s) !=
+        cudaSuccess)
         return FVATTN_ERR_CUDA;
     return FVATTN_OK;
 }
@@ -331,6 +340,7 @@ extern "C" fvattn_status fvattn_route_noalloc(const fvattn_problem *prob, const 
     if (!q || !k || !aligned16(q) || !aligned16(k)) return FVATTN_ERR_INVALID_ARG;
     if (!kv_cnt || !kv_idx || !aligned4(kv_cnt) || !aligned4(kv_idx)) return FVATTN_ERR_INVALID_ARG;
     if (block_probs && !aligned4(block_probs)) return FVATTN_ERR_INVALID_ARG;
+    g.tc_scores = 0;  // the fixed scratch holds no score matrix: scores on the CUDA cores
     const WsLayout L = ws_layout(g);
     const size_t needed = L.kbarT + (size_t)g.BH * g.D * g.nbp * sizeof(float);
     if (needed > kNoAllocScratchBytes) return FVATTN_ERR_WORKSPACE;
@@ -344,8 +354,9 @@ extern "C" fvattn_status fvattn_route_noalloc(const fvattn_problem *prob, const 
     if (launch_pool(g, q, k, reinterpret_cast<float *>(w + L.qbar), reinterpret_cast<float *>(w + L.kbarT), s) !=
         cudaSuccess)
         return FVATTN_ERR_CUDA;
-    if (launch_score_select(g, reinterpret_cast<float *>(w + L.qbar), reinterpret_cast<float *>(w + L.kbarT), p,
-                            k_min, kv_cnt, kv_idx, block_probs, reinterpret_cast<uint32_t *>(w), s) != cudaSuccess)
+    if (launch_score_select(g, reinterpret_cast<float *>(w + L.qbar), reinterpret_cast<float *>(w + L.kbarT),
+                            nullptr, p, k_min, kv_cnt, kv_idx, block_probs, reinterpret_cast<uint32_t *>(w), s) !=
+        cudaSuccess)
         return FVATTN_ERR_CUDA;
     return FVATTN_OK;
 }

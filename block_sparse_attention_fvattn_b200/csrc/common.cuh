@@ -47,6 +47,7 @@ struct Geo {
     int nsub;              // sub-tiles per block along t (2 or 1)
     int rows;              // rows per sub-tile (128 or 64)
     int f16;               // Q, K, V, O are IEEE fp16 (else bf16)
+    int tc_scores;         // routing scores on the tensor cores: pooled K stored [BH, nbp, D], scores in the workspace
     int paired;            // 64-token blocks: two query blocks share one 128-row tile
     int npair;             // pairs of query blocks (2p, 2p+1) per head: ceil(nb/2) when paired
     int upb;               // attention work units per (b, h): nb, or ceil(nb/4) when paired
@@ -76,6 +77,15 @@ struct WsHeader {
 };
 
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Round fp32 to TF32 (10 fraction bits), to nearest with ties away from zero;
+// the result is an fp32 whose 13 low fraction bits are zero.
+__device__ __forceinline__ float tf32_round(float x)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
+}
 
 // ----------------------------------------------------------------------------
 // timing / status

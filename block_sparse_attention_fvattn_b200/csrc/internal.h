@@ -10,8 +10,9 @@ namespace fvattn {
 
 // Workspace carve-up (byte offsets from the workspace base; 256-byte aligned).
 struct WsLayout {
-    size_t qbar;         // fp32 [BH, nb, D]   pooled query means
-    size_t kbarT;        // fp32 [BH, D, nbp]  pooled key means, transposed
+    size_t qbar;         // fp32 [BH, nb, D]   pooled query means ([2][BH, nb, D] TF32 head, rest if tc_scores)
+    size_t kbarT;        // fp32 [BH, D, nbp]  pooled key means, transposed ([2][BH, nbp, D] if tc_scores)
+    size_t scores;       // fp32 [BH, nb, nbp] block scores (tc_scores only)
     size_t unit_cost;    // int32 [BH*nb]      scheduler: cost per unit
     size_t head_sorted;  // int32 [BH*nb]      scheduler: units of each head by cost
     size_t head_cost;    // int64 [BH]         scheduler: total cost per head
@@ -28,9 +29,17 @@ constexpr int kMaxCtas = 4096;
 
 cudaError_t launch_pool(const Geo &g, const void *q, const void *k, float *qbar, float *kbarT,
                         cudaStream_t stream);
-cudaError_t launch_score_select(const Geo &g, const float *qbar, const float *kbarT, float p, int k_min,
-                                int32_t *kv_cnt, int32_t *kv_idx, float *probs, uint32_t *status,
+// scores != nullptr: the block scores were computed by launch_score_gemm.
+cudaError_t launch_score_select(const Geo &g, const float *qbar, const float *kbarT, const float *scores, float p,
+                                int k_min, int32_t *kv_cnt, int32_t *kv_idx, float *probs, uint32_t *status,
                                 cudaStream_t stream);
+// Scores from means split as x = hi + lo (hi, lo exact in TF32), [BH, nb, D]
+// for Q and [BH, nbp, D] for K.
+cudaError_t launch_score_gemm(const Geo &g, const float *qhi, const float *qlo, const float *khi, const float *klo,
+                              float *scores, uint32_t *status, cudaStream_t stream);
+// From this many blocks on, the routing scores run on the tensor cores (at
+// 256 blocks the fused CUDA-core scoring is still faster, at 360 it is slower).
+constexpr int kTcScoresMinBlocks = 320;
 cudaError_t launch_schedule(const Geo &g, const int32_t *kv_cnt, const int32_t *kv_idx, int dense, int num_ctas,
                             int32_t *work, int32_t *cta_range, int64_t *cta_cost, int32_t *unit_cost,
                             int32_t *head_sorted, int64_t *head_cost, const int32_t *pair_cnt,

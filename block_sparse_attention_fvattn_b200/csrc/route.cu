@@ -157,8 +157,19 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geo g, int nxs, cons
         for (int x = xa; x < xb; ++x) sum += red[x * D + d];
         const float mean = sum * (1.0f / (float)(tv * yv * (xb - xa)));
         const int j = (jt * nbh + jy) * nbw + jx0 + jl;
-        if (!which) qbar[((size_t)bh * g.nb + j) * D + d] = mean;
-        else kbarT[((size_t)bh * D + d) * g.nbp + j] = mean;
+        if (g.tc_scores) {
+            // for the tensor cores: [2][BH, rows, D] (rows = nb for Q, nbp for
+            // K), the TF32 head of the mean and then the TF32 head of its rest
+            const float hi = tf32_round(mean), lo = tf32_round(mean - hi);
+            const size_t rows = which ? (size_t)g.nbp : (size_t)g.nb;
+            float *m = which ? kbarT : qbar;
+            m[((size_t)bh * rows + j) * D + d] = hi;
+            m[((size_t)g.BH * rows + (size_t)bh * rows + j) * D + d] = lo;
+        } else if (!which) {
+            qbar[((size_t)bh * g.nb + j) * D + d] = mean;
+        } else {
+            kbarT[((size_t)bh * D + d) * g.nbp + j] = mean;
+        }
     }
 }
 
@@ -478,7 +489,7 @@ __device__ __forceinline__ void score_tile(const float *kb, const float *qsT, fl
 // memory: (D + sel_slices(nbp) * nbp) * ROWS floats.
 template <int D, int EPL>
 __device__ __forceinline__ void select_rows(const Geo &g, int bh, int i0, float *sel_smem,
-                                            const float *qbar, const float *kbarT, float p,
+                                            const float *qbar, const float *kbarT, const float *scores, float p,
                                             int k_min, int32_t *__restrict__ kv_cnt, int32_t *__restrict__ kv_idx,
                                             float *__restrict__ probs, uint32_t *__restrict__ status)
 {
@@ -492,19 +503,27 @@ __device__ __forceinline__ void select_rows(const Geo &g, int bh, int i0, float 
     // scheduler launch behind this grid, then wait for the pooled means
     pdl_release();
     pdl_wait();
-    for (int idx = threadIdx.x; idx < ROWS * D; idx += blockDim.x) {
-        const int r = idx / D, d = idx - r * D;
-        qsT[d * ROWS + r] = (r < nrow) ? qbar[((size_t)bh * g.nb + i0 + r) * D + d] : 0.f;
-    }
-    __syncthreads();
+    if (scores) {
+        // ---- block scores computed on the tensor cores: copy the rows
+        const float4 *src = reinterpret_cast<const float4 *>(scores + ((size_t)bh * g.nb + i0) * nbp);
+        float4 *dst = reinterpret_cast<float4 *>(sc);
+        const int n4 = nrow * nbp / 4;
+        for (int x = threadIdx.x; x < n4; x += blockDim.x) dst[x] = __ldcg(src + x);
+    } else {
+        for (int idx = threadIdx.x; idx < ROWS * D; idx += blockDim.x) {
+            const int r = idx / D, d = idx - r * D;
+            qsT[d * ROWS + r] = (r < nrow) ? qbar[((size_t)bh * g.nb + i0 + r) * D + d] : 0.f;
+        }
+        __syncthreads();
 
-    // ---- block scores
-    const float *kb = kbarT + (size_t)bh * D * nbp;
-    const int S = sel_slices(nbp);
-    if (S == 8) score_tile<D, 8, ROWS>(kb, qsT, sc, nbp, g.scale);
-    else if (S == 4) score_tile<D, 4, ROWS>(kb, qsT, sc, nbp, g.scale);
-    else if (S == 2) score_tile<D, 2, ROWS>(kb, qsT, sc, nbp, g.scale);
-    else score_tile<D, 1, ROWS>(kb, qsT, sc, nbp, g.scale);
+        // ---- block scores
+        const float *kb = kbarT + (size_t)bh * D * nbp;
+        const int S = sel_slices(nbp);
+        if (S == 8) score_tile<D, 8, ROWS>(kb, qsT, sc, nbp, g.scale);
+        else if (S == 4) score_tile<D, 4, ROWS>(kb, qsT, sc, nbp, g.scale);
+        else if (S == 2) score_tile<D, 2, ROWS>(kb, qsT, sc, nbp, g.scale);
+        else score_tile<D, 1, ROWS>(kb, qsT, sc, nbp, g.scale);
+    }
     __syncthreads();
 
     // ---- selection: one warp per row
@@ -664,12 +683,13 @@ __device__ __forceinline__ void select_rows(const Geo &g, int bh, int i0, float 
 template <int D, int EPL>
 __global__ void __launch_bounds__(256, kSelMinBlocksFor<EPL>) score_select_kernel(Geo g, const float *__restrict__ qbar,
                                                            const float *__restrict__ kbarT, float p, int k_min,
+                                                           const float *__restrict__ scores,
                                                            int32_t *__restrict__ kv_cnt, int32_t *__restrict__ kv_idx,
                                                            float *__restrict__ probs, uint32_t *__restrict__ status)
 {
     extern __shared__ __align__(16) float sel_smem[];
-    select_rows<D, EPL>(g, blockIdx.y, blockIdx.x * kSelRowsFor<EPL>, sel_smem, qbar, kbarT, p, k_min, kv_cnt, kv_idx, probs,
-                        status);
+    select_rows<D, EPL>(g, blockIdx.y, blockIdx.x * kSelRowsFor<EPL>, sel_smem, qbar, kbarT, scores, p, k_min, kv_cnt,
+                        kv_idx, probs, status);
 }
 
 // ---------------------------------------------------------------------------
@@ -717,8 +737,8 @@ cudaError_t launch_pool(const Geo &g, const void *q, const void *k, float *qbar,
 }
 
 template <int D, int EPL>
-static cudaError_t launch_sel_t(const Geo &g, const float *qbar, const float *kbarT, float p, int k_min,
-                                int32_t *kv_cnt, int32_t *kv_idx, float *probs, uint32_t *status,
+static cudaError_t launch_sel_t(const Geo &g, const float *qbar, const float *kbarT, const float *scores, float p,
+                                int k_min, int32_t *kv_cnt, int32_t *kv_idx, float *probs, uint32_t *status,
                                 cudaStream_t stream)
 {
     constexpr int ROWS = kSelRowsFor<EPL>;
@@ -730,17 +750,17 @@ static cudaError_t launch_sel_t(const Geo &g, const float *qbar, const float *kb
     // programmatic dependent launch: the CTAs may be scheduled while the
     // pooling kernel drains and wait in-kernel for its results
     return launch_dependent(kern, dim3((unsigned)ceil_div(g.nb, ROWS), (unsigned)g.BH), dim3(256), smem, stream, g,
-                            qbar, kbarT, p, k_min, kv_cnt, kv_idx, probs, status);
+                            qbar, kbarT, p, k_min, scores, kv_cnt, kv_idx, probs, status);
 }
 
 template <int D>
-static cudaError_t launch_sel_d(const Geo &g, const float *qbar, const float *kbarT, float p, int k_min,
-                                int32_t *kv_cnt, int32_t *kv_idx, float *probs, uint32_t *status,
+static cudaError_t launch_sel_d(const Geo &g, const float *qbar, const float *kbarT, const float *scores, float p,
+                                int k_min, int32_t *kv_cnt, int32_t *kv_idx, float *probs, uint32_t *status,
                                 cudaStream_t stream)
 {
     const int epl = ceil_div(g.nb, 32);
 #define FV_SEL(E) \
-    if (epl <= E) return launch_sel_t<D, E>(g, qbar, kbarT, p, k_min, kv_cnt, kv_idx, probs, status, stream)
+    if (epl <= E) return launch_sel_t<D, E>(g, qbar, kbarT, scores, p, k_min, kv_cnt, kv_idx, probs, status, stream)
     FV_SEL(1);
     FV_SEL(2);
     FV_SEL(4);
@@ -755,12 +775,12 @@ static cudaError_t launch_sel_d(const Geo &g, const float *qbar, const float *kb
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_score_select(const Geo &g, const float *qbar, const float *kbarT, float p, int k_min,
-                                int32_t *kv_cnt, int32_t *kv_idx, float *probs, uint32_t *status,
+cudaError_t launch_score_select(const Geo &g, const float *qbar, const float *kbarT, const float *scores, float p,
+                                int k_min, int32_t *kv_cnt, int32_t *kv_idx, float *probs, uint32_t *status,
                                 cudaStream_t stream)
 {
-    if (g.D == 128) return launch_sel_d<128>(g, qbar, kbarT, p, k_min, kv_cnt, kv_idx, probs, status, stream);
-    return launch_sel_d<64>(g, qbar, kbarT, p, k_min, kv_cnt, kv_idx, probs, status, stream);
+    if (g.D == 128) return launch_sel_d<128>(g, qbar, kbarT, scores, p, k_min, kv_cnt, kv_idx, probs, status, stream);
+    return launch_sel_d<64>(g, qbar, kbarT, scores, p, k_min, kv_cnt, kv_idx, probs, status, stream);
 }
 
 }  // namespace fvattn

@@ -23,8 +23,9 @@ TOPP_WINDOW = 1e-5
 # Rounding-tie window for list differences at the rank boundary: the fp32
 # pooled scores can differ from the fp64 ones by at most about
 # (D + 2*256) * 2^-24 * scale * |Qbar_i| * |Kbar_j| (dot-product and pooled-sum
-# error bounds), so two blocks whose oracle scores are closer than that may
-# legitimately swap ranks.
+# error bounds; the three-product TF32 split used for long rows adds at most
+# 3 * 2^-22 of the same scale), so two blocks whose oracle scores are closer
+# than that may legitimately swap ranks.
 TIE_FACTOR = 4e-5
 
 
