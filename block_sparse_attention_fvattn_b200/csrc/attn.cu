@@ -25,13 +25,14 @@
 // article, section 5.1, on n x n masks at ~400k tokens).
 //
 // Roles (384 threads = 3 warpgroups, one CTA per SM):
-//   warp 0      TMA producer of Q halves and K sub-tiles; takes the units
+//   warp 0      TMA producer of Q halves and K sub-tiles
 //   warp 1      QK issuer (one thread) and owner of the TMEM allocation:
 //               S = Q_h K^T (A and B from shared memory)
 //   warp 2      PV issuer (one thread): O_h += P_h V (A = P_h from TMEM,
 //               B = V from shared memory, MN-major). Two issuing threads keep
 //               the tensor core fed while either one waits on a barrier.
-//   warp 3      TMA producer of V sub-tiles (follows warp 0's units)
+//   warp 3      TMA producer of V sub-tiles; its lane 1 takes the units from
+//               the shared counter, one unit ahead of warp 0
 //   warps 4-7   softmax + epilogue for query half 0
 //   warps 8-11  softmax + epilogue for query half 1
 // A warp reaches TMEM lanes 32*(warp % 4) .. +31, so each softmax warpgroup
@@ -44,6 +45,16 @@
 // registers, so the next QK never waits for a PV to finish, and one half's
 // softmax overlaps the other half's products. The online softmax rescales O
 // lazily, only when a row maximum grows by more than 2^8.
+//
+// Epilogue: O / l is staged in the half's Q tile (whose products are all done
+// by then), in that tile's swizzled layout, and written by TMA tile stores
+// with the same 5-D boxes as the loads, so rows outside the grid are skipped
+// and every store is a whole 128-byte line. The next unit's Q tile is loaded
+// there once the stores have read it.
+// Units: lane 1 of warp 3 claims them from the counter shared by all CTAs, one
+// unit ahead of warp 0. A slot of the unit ring carries the unit id and, in
+// paired mode, the two union sizes and the first entries of each union, so no
+// role starts a unit with a chain of global loads.
 #include "common.cuh"
 #include "exp2_poly.h"
 #include "internal.h"
@@ -59,7 +70,11 @@
 
 namespace fvattn {
 
-constexpr int kUnitSlots = 4;  // ring of unit ids handed from the producer to the other roles
+constexpr int kUnitSlots = 4;  // ring of units handed from the producer to the other roles
+// words of a unit slot: the unit id, then (paired mode) the two union sizes and
+// the first two entries of each union, so no role reads them from global
+// memory at the start of a unit
+constexpr int kUnitWords = 8;
 constexpr int kThreads = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Register split between warpgroups (setmaxnreg). The kernel is launched with
@@ -94,19 +109,21 @@ struct AttnLayout {
     // per-axis column masks: entry v-1 of each axis keeps the columns whose
     // coordinate along that axis is < v; blk_w + blk_h + sub_t <= kMaskEntries
     static constexpr int kMaskEntries = 40;
-    static constexpr int kUnit = kMask + kMaskEntries * kMaskWords * 4;  // int32 unit ids
-    static constexpr int kBar = kUnit + 8 * ((kUnitSlots * 4 + 7) / 8);
+    static constexpr int kUnit = kMask + kMaskEntries * kMaskWords * 4;  // int32 unit slots
+    static constexpr int kBar = kUnit + kUnitSlots * kUnitWords * 4;
     // barrier indices
     static constexpr int bQFull = 0, bQEmpty = 2, bKFull = 4, bKEmpty = bKFull + kNK, bVFull = bKEmpty + kNK,
                          bVEmpty = bVFull + kNV, bSFull = bVEmpty + kNV, bSFree = bSFull + 2, bPFull = bSFree + 1,
                          bPFree = bPFull + 2, bOFull = bPFree + 2, bOEmpty = bOFull + 2, bDrain = bOEmpty + 2,
-                         bUFull = bDrain + 2, bUEmpty = bUFull + kUnitSlots, kNumBars = bUEmpty + kUnitSlots;
-    // arrivals that free a unit slot: the V producer, the QK and PV issuers and
-    // the 8 softmax warps
-    static constexpr int kUnitConsumers = 11;
+                         bUFull = bDrain + 2, bUEmpty = bUFull + kUnitSlots, bOStaged = bUEmpty + kUnitSlots,
+                         bTaken = bOStaged + 2, kNumBars = bTaken + 1;
+    // arrivals that free a unit slot: the two producers, the QK and PV issuers
+    // and the 8 softmax warps
+    static constexpr int kUnitConsumers = 12;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 64;
     static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
+    static_assert(kAlloc <= 227 * 1024, "shared memory per CTA");
     // TMEM columns
     static constexpr uint32_t kTmS = 0, kTmP = 128, kTmO = 256;
     static uint32_t __device__ __forceinline__ tm_p(int h) { return kTmP + 64u * (uint32_t)h; }
@@ -213,6 +230,21 @@ __device__ __forceinline__ PairUnit load_pair_unit(const Geo &g, int u, const in
     return P;
 }
 
+// The same from the union sizes published in the unit ring (no loads).
+__device__ __forceinline__ PairUnit pair_unit_from(const Geo &g, int u, int c0, int c1, const int32_t *pair_list,
+                                                   int dense)
+{
+    PairUnit P;
+    P.bh = u / g.upb;
+    P.q = u - P.bh * g.upb;
+    P.c0 = c0;
+    P.c1 = c1;
+    const size_t pid = (size_t)P.bh * g.npair + 2 * P.q;
+    P.l0 = (dense || c0 == 0) ? nullptr : pair_list + pid * g.nb;
+    P.l1 = (dense || c1 == 0) ? nullptr : pair_list + (pid + 1) * g.nb;
+    return P;
+}
+
 // Entry e of a union of c entries. Past the end (the second block of an odd
 // last tile) it repeats the last block with no keeper, so that block's
 // columns are masked out for every row.
@@ -238,7 +270,8 @@ __device__ __forceinline__ int rank_to_unit(long long r, const int32_t *work, co
 }
 
 // Consumer side of the unit ring: wait for the n-th slot and read its unit id
-// (-1 ends the sequence). The caller frees the slot once it has read it.
+// (-1 ends the sequence); meta() reads the slot's other words. The caller
+// frees the slot once it has read what it needs.
 struct UnitFeed {
     uint32_t full0;
     const volatile int32_t *slots;
@@ -251,8 +284,9 @@ struct UnitFeed {
             return -1;
         }
         ++n;
-        return slots[slot];
+        return slots[slot * kUnitWords];
     }
+    __device__ __forceinline__ int meta(int slot, int i) const { return slots[slot * kUnitWords + i]; }
 };
 
 // Two exponentials 2^a (a = packed pair) on the FMA/ALU pipes:
@@ -283,10 +317,10 @@ __device__ __forceinline__ void exp2_poly_x2(uint64_t a, float &p0, float &p1)
 template <int D, int BKV, bool PAIRED, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, Geo g, const int32_t *__restrict__ kv_cnt,
-                const int32_t *__restrict__ kv_idx, const int32_t *__restrict__ pair_cnt,
-                const int32_t *__restrict__ pair_list, const int32_t *__restrict__ work,
-                const int32_t *__restrict__ cta_range, int dense, uint16_t *__restrict__ out,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, Geo g,
+                const int32_t *__restrict__ kv_cnt, const int32_t *__restrict__ kv_idx,
+                const int32_t *__restrict__ pair_cnt, const int32_t *__restrict__ pair_list,
+                const int32_t *__restrict__ work, const int32_t *__restrict__ cta_range, int dense,
                 int64_t *__restrict__ cta_ns, uint32_t *__restrict__ status)
 {
     static_assert(!PAIRED || BKV == 128, "paired mode runs 128-token key/value tiles");
@@ -326,7 +360,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         for (int b = 0; b < L::kNumBars; ++b) {
             uint32_t cnt = 1;
-            if (b == L::bSFree || b == L::bPFull || b == L::bPFull + 1 || b == L::bOEmpty || b == L::bOEmpty + 1)
+            if (b == L::bSFree || b == L::bPFull || b == L::bPFull + 1 || b == L::bOEmpty || b == L::bOEmpty + 1 ||
+                b == L::bOStaged || b == L::bOStaged + 1)
                 cnt = 128;  // arrived on by all 128 threads of a softmax warpgroup
             if (b >= L::bUEmpty && b < L::bUEmpty + kUnitSlots) cnt = L::kUnitConsumers;
             mbar_init(bar(b), cnt);
@@ -359,11 +394,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t q_bytes = (uint32_t)L::kDH * (uint32_t)g.rows * 128u;
 
     if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(RegSplit<D, BKV>::kLow));
-    if (warp == 0 || warp == 3) {
+    if (warp == 3 && lane == 1) {
+        // ================= unit claimer =================
+        // Slot n of the unit ring: the unit id and, paired, its union sizes and
+        // first entries. Unit n is claimed once warp 0 has taken unit n-1, so
+        // the claim's chain of loads hides behind that unit while the dynamic
+        // longest-first order keeps a lookahead of one unit.
+        bool ok = true;
+        for (int n = 0; ok; ++n) {
+            const int slot = n % kUnitSlots;
+            if (n > 0 && !mbar_wait(bar(L::bTaken), (uint32_t)(n - 1) & 1u, abort_flag)) break;
+            if (n >= kUnitSlots &&
+                !mbar_wait(bar(L::bUEmpty + slot), (uint32_t)((n / kUnitSlots) - 1) & 1u, abort_flag))
+                break;
+            const long long r = (long long)atomicAdd(unit_cursor, 1u);
+            const int u = r < n_units ? rank_to_unit(r, work, cta_range) : -1;
+            int m[kUnitWords];
+            m[0] = u;
+#pragma unroll
+            for (int i = 1; i < kUnitWords; ++i) m[i] = 0;
+            if (PAIRED && u >= 0) {
+                const PairUnit P = load_pair_unit(g, u, pair_cnt, pair_list, dense);
+                m[1] = P.c0;
+                m[2] = P.c1;
+                m[3] = pair_entry(P.l0, P.c0, 0);
+                m[4] = pair_entry(P.l0, P.c0, 1);
+                m[5] = pair_entry(P.l1, P.c1, 0);
+                m[6] = pair_entry(P.l1, P.c1, 1);
+            }
+#pragma unroll
+            for (int i = 0; i < kUnitWords; ++i) unit_slots[slot * kUnitWords + i] = m[i];
+            mbar_arrive(bar(L::bUFull + slot));  // release: the slot is visible to the waiting roles
+            if (u < 0) break;
+        }
+    } else if (warp == 0 || warp == 3) {
         // ================= TMA producers =================
-        // warp 0 takes the units and loads Q and K; warp 3 follows the same
-        // units (through the unit ring) and loads V, so a K load never waits
-        // for a V slot, which frees only after a softmax and a PV
+        // warp 0 loads Q and K; warp 3 loads V for the same units, so a K load
+        // never waits for a V slot, which frees only after a softmax and a PV
         if (lane == 0) {
             const bool vrole = warp == 3;
             if (vrole) {
@@ -424,27 +491,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return true;
             };
             for (int n = 0; ok; ++n) {
-                int u;
-                if (!vrole) {
-                    const int slot = n % kUnitSlots;
-                    if (n >= kUnitSlots &&
-                        !mbar_wait(bar(L::bUEmpty + slot), (uint32_t)((n / kUnitSlots) - 1) & 1u, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    const long long r = (long long)atomicAdd(unit_cursor, 1u);
-                    u = r < n_units ? rank_to_unit(r, work, cta_range) : -1;
-                    unit_slots[slot] = u;
-                    mbar_arrive(bar(L::bUFull + slot));  // release: the id is visible to the waiting roles
-                } else {
+                int um[kUnitWords];
+                {
                     int slot;
-                    u = feed.next(abort_flag, ok, slot);
+                    um[0] = feed.next(abort_flag, ok, slot);
                     if (!ok) break;
+#pragma unroll
+                    for (int i = 1; i < kUnitWords; ++i) um[i] = feed.meta(slot, i);
                     mbar_arrive(bar(L::bUEmpty + slot));
+                    if (!vrole) mbar_arrive(bar(L::bTaken));  // the claimer may take the next unit
                 }
+                const int u = um[0];
                 if (u < 0) break;
                 if constexpr (PAIRED) {
-                    const PairUnit P = load_pair_unit(g, u, pair_cnt, pair_list, dense);
+                    const PairUnit P = pair_unit_from(g, u, um[1], um[2], pair_list, dense);
                     for (int h = 0; h < 2 && ok && !vrole; ++h) {
                         if (P.cnt(h) == 0) continue;
                         const int qa = 2 * (2 * P.q + h);  // rows 0-63: block qa, rows 64-127: block qa+1
@@ -454,8 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // half 0, then tile r of half 1 (each while that half has one)
                     const int rounds = max(P.tiles(0), P.tiles(1));
                     // a round's four entries are loaded one round ahead
-                    int cur[4] = {pair_entry(P.l0, P.c0, 0), pair_entry(P.l0, P.c0, 1), pair_entry(P.l1, P.c1, 0),
-                                  pair_entry(P.l1, P.c1, 1)};
+                    int cur[4] = {um[3], um[4], um[5], um[6]};
                     for (int r = 0; r < rounds && ok; ++r) {
                         const int nxt[4] = {pair_entry(P.l0, P.c0, 2 * r + 2), pair_entry(P.l0, P.c0, 2 * r + 3),
                                             pair_entry(P.l1, P.c1, 2 * r + 2), pair_entry(P.l1, P.c1, 2 * r + 3)};
@@ -517,19 +576,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int slot;
                 const int u = feed.next(abort_flag, ok, slot);
                 if (!ok) break;
+                const int mc0 = feed.meta(slot, 1), mc1 = feed.meta(slot, 2);
                 mbar_arrive(bar(L::bUEmpty + slot));
                 if (u < 0) break;
                 if constexpr (PAIRED) {
-                    const PairUnit P = load_pair_unit(g, u, pair_cnt, pair_list, dense);
-                    for (int h = 0; h < 2 && ok; ++h) {
-                        if (P.cnt(h) == 0) continue;
-                        ok = mbar_wait(bar(L::bQFull + h), (ph_q >> h) & 1u, abort_flag);
-                        ph_q ^= 1u << h;
-                    }
+                    const PairUnit P = pair_unit_from(g, u, mc0, mc1, pair_list, dense);
                     const int rounds = max(P.tiles(0), P.tiles(1));
                     for (int r = 0; r < rounds && ok; ++r) {
                         for (int h = 0; h < 2 && ok; ++h) {
                             if (r >= P.tiles(h)) continue;
+                            // each half's Q tile is waited for just before its first product
+                            if (r == 0) {
+                                ok = mbar_wait(bar(L::bQFull + h), (ph_q >> h) & 1u, abort_flag);
+                                ph_q ^= 1u << h;
+                                if (!ok) break;
+                            }
                             const int ks = kc % L::kNK;
                             if (!mbar_wait(bar(L::bKFull + ks), (kc / L::kNK) & 1, abort_flag)) { ok = false; break; }
                             if (qk_count > 0 && !mbar_wait(bar(L::bSFree), (qk_count - 1) & 1, abort_flag)) {
@@ -540,7 +601,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                             issue_qk(h, ks);
                             umma_commit(bar(L::bSFull + h));
                             ++qk_count;
-                            if (r == P.tiles(h) - 1) umma_commit(bar(L::bQEmpty + h));
                             umma_commit(bar(L::bKEmpty + ks));
                             ++kc;
                         }
@@ -566,7 +626,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         issue_qk(h, ks);
                         umma_commit(bar(L::bSFull + h));
                         ++qk_count;
-                        if (k == U.nkv - 1) umma_commit(bar(L::bQEmpty + h));
                     }
                     if (!ok) break;
                     umma_commit(bar(L::bKEmpty + ks));
@@ -608,10 +667,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int slot;
                 const int u = feed.next(abort_flag, ok, slot);
                 if (!ok) break;
+                const int mc0 = feed.meta(slot, 1), mc1 = feed.meta(slot, 2);
                 mbar_arrive(bar(L::bUEmpty + slot));
                 if (u < 0) break;
                 if constexpr (PAIRED) {
-                    const PairUnit P = load_pair_unit(g, u, pair_cnt, pair_list, dense);
+                    const PairUnit P = pair_unit_from(g, u, mc0, mc1, pair_list, dense);
                     const int rounds = max(P.tiles(0), P.tiles(1));
                     for (int r = 0; r < rounds && ok; ++r) {
                         for (int h = 0; h < 2 && ok; ++h) {
@@ -671,10 +731,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tP = tmem + t_lane + L::tm_p(h);
         const uint32_t tO = tmem + t_lane + L::tm_o(h);
         const float sl2 = g.scale * 1.4426950408889634f;
-        // this thread's query row inside a sub-tile (paired mode: inside its
-        // 64-token query block, which is the first of the pair for rows 0-63)
-        const int r64 = PAIRED ? (row & 63) : row;
-        const int r_t = r64 / (g.bh * g.bw), r_y = (r64 / g.bw) % g.bh, r_x = r64 % g.bw;
         int sf = 0, of = 0, pw = 0;  // S tiles received, O tiles received, P tiles written
         bool ok = true;
         float m = -INFINITY, l = 0.f;
@@ -789,58 +845,83 @@ __global__ void __launch_bounds__(kThreads, 1)
             l += sum;
             return true;
         };
-        // epilogue: O / l -> bf16, raster order, valid rows only
-        auto epilogue = [&](int ubh, int qt, int qy, int qx, bool row_valid) -> bool {
+        // epilogue: O / l in the element type, staged in this half's Q tile (every
+        // product that reads it is done once O_h is complete) in the tile's own
+        // swizzled layout, then written by TMA stores, which skip the rows
+        // outside the grid; the Q tile goes back to the producer once the stores
+        // have read it
+        const uint32_t o_stage = sbase + L::kQ + (uint32_t)(h * L::kDH * L::kQSlab) + (uint32_t)row * 128u;
+        auto epilogue = [&](int ubh, int i0, int nblk, int t_off) -> bool {
             if (!mbar_wait(bar(L::bOFull + h), of & 1, abort_flag)) return false;
             ++of;
             tc_fence_after();
             const float inv = 1.0f / l;
-            uint16_t *orow =
-                out + ((size_t)ubh * g.N + ((size_t)qt * g.Hg + qy) * g.W + qx) * (size_t)D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
                 tmem_ld32(tO + c * 32, o);
                 tmem_wait_ld();
-                if (row_valid) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+                if (c == D / 32 - 1) {
+                    // O_h has been read: the next unit's first product may overwrite it
+                    tc_fence_before();
+                    mbar_arrive(bar(L::bOEmpty + h));
+                }
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint4 w;
-                        w.x = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 0]) * inv, __uint_as_float(o[q4 * 8 + 1]) * inv);
-                        w.y = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 2]) * inv, __uint_as_float(o[q4 * 8 + 3]) * inv);
-                        w.z = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 4]) * inv, __uint_as_float(o[q4 * 8 + 5]) * inv);
-                        w.w = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 6]) * inv, __uint_as_float(o[q4 * 8 + 7]) * inv);
-                        dst[q4] = w;
-                    }
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint4 w;
+                    w.x = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 0]) * inv, __uint_as_float(o[q4 * 8 + 1]) * inv);
+                    w.y = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 2]) * inv, __uint_as_float(o[q4 * 8 + 3]) * inv);
+                    w.z = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 4]) * inv, __uint_as_float(o[q4 * 8 + 5]) * inv);
+                    w.w = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 6]) * inv, __uint_as_float(o[q4 * 8 + 7]) * inv);
+                    // 16-byte piece j of the row: slab j / 8, 128-byte swizzle of piece j % 8
+                    const int j = c * 4 + q4;
+                    st_shared_v4(o_stage + (uint32_t)((j >> 3) * L::kQSlab) + (uint32_t)(((j & 7) ^ (row & 7)) << 4),
+                                 w);
                 }
             }
-            tc_fence_before();
-            mbar_arrive(bar(L::bOEmpty + h));
+            // the tile is written: make it visible to the TMA engine, then the
+            // storing thread waits (with the usual time limit) for all 128 rows
+            fence_proxy_async();
+            mbar_arrive(bar(L::bOStaged + h));
+            if (row == 0) {
+                if (!mbar_wait(bar(L::bOStaged + h), (of - 1) & 1, abort_flag)) return false;
+                for (int s2 = 0; s2 < nblk; ++s2) {
+                    int jt, jy, jx;
+                    block_coords(g, i0 + s2, jt, jy, jx);
+                    for (int dh = 0; dh < L::kDH; ++dh)
+                        tma_store_5d(&tm_o, sbase + L::kQ + (h * L::kDH + dh) * L::kQSlab + s2 * kHalfRows, dh * 64,
+                                     jx * g.bw, jy * g.bh, jt * g.bt + t_off, ubh);
+                }
+                bulk_commit_group();
+                bulk_wait_read_all();
+                mbar_arrive(bar(L::bQEmpty + h));
+            }
             return true;
         };
         while (ok) {
             int slot;
             const int u = feed.next(abort_flag, ok, slot);
             if (!ok) break;
+            int mc0 = 0, mc1 = 0, me0 = 0, me1 = 0;
+            if constexpr (PAIRED) {
+                mc0 = feed.meta(slot, 1);
+                mc1 = feed.meta(slot, 2);
+                me0 = feed.meta(slot, 3 + 2 * h);
+                me1 = feed.meta(slot, 4 + 2 * h);
+            }
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(L::bUEmpty + slot));  // every lane has read the id
+            if (lane == 0) mbar_arrive(bar(L::bUEmpty + slot));  // every lane has read the slot
             if (u < 0) break;
             if constexpr (PAIRED) {
-                const PairUnit P = load_pair_unit(g, u, pair_cnt, pair_list, dense);
+                const PairUnit P = pair_unit_from(g, u, mc0, mc1, pair_list, dense);
                 const int c_h = P.cnt(h), n_h = P.tiles(h);
                 const int32_t *lst = P.list(h);
                 if (n_h == 0) continue;
                 const int hb = row >> 6;                   // 0: first query block of the pair, 1: second
-                const int qi = 2 * (2 * P.q + h) + hb;     // this row's query block
                 const int keeper = hb ? kPairInB : kPairInA;
-                int it, iy, ix;
-                block_coords(g, qi, it, iy, ix);
-                const int qt = it * g.bt + r_t, qy = iy * g.bh + r_y, qx = ix * g.bw + r_x;
-                const bool row_valid = qi < g.nb && qt < g.T && qy < g.Hg && qx < g.W;
                 m = -INFINITY;
                 l = 0.f;
-                int ent0 = pair_entry(lst, c_h, 0), ent1 = pair_entry(lst, c_h, 1);
+                int ent0 = me0, ent1 = me1;
                 for (int r = 0; r < n_h; ++r) {
                     // the next tile's entries are loaded now and used next iteration
                     const int nxt0 = pair_entry(lst, c_h, 2 * r + 2), nxt1 = pair_entry(lst, c_h, 2 * r + 3);
@@ -881,13 +962,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ent1 = nxt1;
                 }
                 if (!ok) break;
-                if (!epilogue(P.bh, qt, qy, qx, row_valid)) { ok = false; break; }
+                const int qa = 2 * (2 * P.q + h);
+                if (!epilogue(P.bh, qa, qa + 1 < g.nb ? 2 : 1, 0)) { ok = false; break; }
                 continue;
             }
             const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
             if (h >= U.nh) continue;
-            const int qt = U.it * g.bt + h * g.subt + r_t, qy = U.iy * g.bh + r_y, qx = U.ix * g.bw + r_x;
-            const bool row_valid = row < g.rows && qt < g.T && qy < g.Hg && qx < g.W;
             m = -INFINITY;
             l = 0.f;
             int e = 0, s_sub = 0;
@@ -923,8 +1003,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (!ok) break;
-            if (!epilogue(U.bh, qt, qy, qx, row_valid)) { ok = false; break; }
+            if (!epilogue(U.bh, U.i, 1, h * g.subt)) { ok = false; break; }
         }
+        // the output stores have completed before the CTA exits
+        if (row == 0) bulk_wait_all();
     }
 
     tc_fence_before();
@@ -983,9 +1065,10 @@ static bool make_map(CUtensorMap *map, const Geo &g, const void *ptr)
 
 template <int D, int BKV, bool PAIRED, bool F16>
 static cudaError_t launch_attn_f(const Geo &g, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
-                                 const int32_t *kv_cnt, const int32_t *kv_idx, const int32_t *pair_cnt,
-                                 const int32_t *pair_list, const int32_t *work, const int32_t *cta_range, int grid,
-                                 int dense, void *out, int64_t *cta_ns, uint32_t *status, cudaStream_t stream)
+                                 const CUtensorMap &mo, const int32_t *kv_cnt, const int32_t *kv_idx,
+                                 const int32_t *pair_cnt, const int32_t *pair_list, const int32_t *work,
+                                 const int32_t *cta_range, int grid, int dense, int64_t *cta_ns, uint32_t *status,
+                                 cudaStream_t stream)
 {
     using L = AttnLayout<D, BKV, PAIRED>;
     auto kern = attn_kernel<D, BKV, PAIRED, F16>;
@@ -998,21 +1081,22 @@ static cudaError_t launch_attn_f(const Geo &g, const CUtensorMap &mq, const CUte
         return cudaErrorInvalidConfiguration;
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (err != cudaSuccess) return err;
-    return launch_dependent(kern, dim3(grid), dim3(kThreads), L::kAlloc, stream, mq, mk, mv, g, kv_cnt, kv_idx,
-                            pair_cnt, pair_list, work, cta_range, dense, (uint16_t *)out, cta_ns, status);
+    return launch_dependent(kern, dim3(grid), dim3(kThreads), L::kAlloc, stream, mq, mk, mv, mo, g, kv_cnt, kv_idx,
+                            pair_cnt, pair_list, work, cta_range, dense, cta_ns, status);
 }
 
 template <int D, int BKV, bool PAIRED>
 static cudaError_t launch_attn_t(const Geo &g, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
-                                 const int32_t *kv_cnt, const int32_t *kv_idx, const int32_t *pair_cnt,
-                                 const int32_t *pair_list, const int32_t *work, const int32_t *cta_range, int grid,
-                                 int dense, void *out, int64_t *cta_ns, uint32_t *status, cudaStream_t stream)
+                                 const CUtensorMap &mo, const int32_t *kv_cnt, const int32_t *kv_idx,
+                                 const int32_t *pair_cnt, const int32_t *pair_list, const int32_t *work,
+                                 const int32_t *cta_range, int grid, int dense, int64_t *cta_ns, uint32_t *status,
+                                 cudaStream_t stream)
 {
     if (g.f16)
-        return launch_attn_f<D, BKV, PAIRED, true>(g, mq, mk, mv, kv_cnt, kv_idx, pair_cnt, pair_list, work,
-                                                   cta_range, grid, dense, out, cta_ns, status, stream);
-    return launch_attn_f<D, BKV, PAIRED, false>(g, mq, mk, mv, kv_cnt, kv_idx, pair_cnt, pair_list, work, cta_range,
-                                                grid, dense, out, cta_ns, status, stream);
+        return launch_attn_f<D, BKV, PAIRED, true>(g, mq, mk, mv, mo, kv_cnt, kv_idx, pair_cnt, pair_list, work,
+                                                   cta_range, grid, dense, cta_ns, status, stream);
+    return launch_attn_f<D, BKV, PAIRED, false>(g, mq, mk, mv, mo, kv_cnt, kv_idx, pair_cnt, pair_list, work,
+                                                cta_range, grid, dense, cta_ns, status, stream);
 }
 
 cudaError_t launch_attn(const Geo &g, const void *q, const void *k, const void *v, const int32_t *kv_cnt,
@@ -1021,8 +1105,8 @@ cudaError_t launch_attn(const Geo &g, const void *q, const void *k, const void *
                         int64_t *cta_ns, uint32_t *status, cudaStream_t stream, int *launch_error_kind)
 {
     *launch_error_kind = 0;
-    CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, g, q) || !make_map(&mk, g, k) || !make_map(&mv, g, v)) {
+    CUtensorMap mq, mk, mv, mo;
+    if (!make_map(&mq, g, q) || !make_map(&mk, g, k) || !make_map(&mv, g, v) || !make_map(&mo, g, out)) {
         *launch_error_kind = 1;
         return cudaErrorInvalidValue;
     }
@@ -1033,16 +1117,16 @@ cudaError_t launch_attn(const Geo &g, const void *q, const void *k, const void *
     }
     if (g.paired) {
         if (g.D == 128)
-            return launch_attn_t<128, 128, true>(g, mq, mk, mv, kv_cnt, kv_idx, pair_cnt, pair_list, work, cta_range,
-                                                 grid, dense, out, cta_ns, status, stream);
-        return launch_attn_t<64, 128, true>(g, mq, mk, mv, kv_cnt, kv_idx, pair_cnt, pair_list, work, cta_range,
-                                            grid, dense, out, cta_ns, status, stream);
+            return launch_attn_t<128, 128, true>(g, mq, mk, mv, mo, kv_cnt, kv_idx, pair_cnt, pair_list, work,
+                                                 cta_range, grid, dense, cta_ns, status, stream);
+        return launch_attn_t<64, 128, true>(g, mq, mk, mv, mo, kv_cnt, kv_idx, pair_cnt, pair_list, work,
+                                            cta_range, grid, dense, cta_ns, status, stream);
     }
     if (g.D == 128)
-        return launch_attn_t<128, 128, false>(g, mq, mk, mv, kv_cnt, kv_idx, pair_cnt, pair_list, work, cta_range,
-                                              grid, dense, out, cta_ns, status, stream);
-    return launch_attn_t<64, 128, false>(g, mq, mk, mv, kv_cnt, kv_idx, pair_cnt, pair_list, work, cta_range, grid,
-                                         dense, out, cta_ns, status, stream);
+        return launch_attn_t<128, 128, false>(g, mq, mk, mv, mo, kv_cnt, kv_idx, pair_cnt, pair_list, work,
+                                              cta_range, grid, dense, cta_ns, status, stream);
+    return launch_attn_t<64, 128, false>(g, mq, mk, mv, mo, kv_cnt, kv_idx, pair_cnt, pair_list, work,
+                                         cta_range, grid, dense, cta_ns, status, stream);
 }
 
 }  // namespace fvattn
