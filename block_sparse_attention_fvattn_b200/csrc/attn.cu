@@ -32,7 +32,7 @@
 //               B = V from shared memory, MN-major). Two issuing threads keep
 //               the tensor core fed while either one waits on a barrier.
 //   warp 3      TMA producer of V sub-tiles; its lane 1 takes the units from
-//               the shared counter, one unit ahead of warp 0
+//               the shared counter once warp 0 has issued the current unit
 //   warps 4-7   softmax + epilogue for query half 0
 //   warps 8-11  softmax + epilogue for query half 1
 // A warp reaches TMEM lanes 32*(warp % 4) .. +31, so each softmax warpgroup
@@ -51,8 +51,8 @@
 // with the same 5-D boxes as the loads, so rows outside the grid are skipped
 // and every store is a whole 128-byte line. The next unit's Q tile is loaded
 // there once the stores have read it.
-// Units: lane 1 of warp 3 claims them from the counter shared by all CTAs, one
-// unit ahead of warp 0. A slot of the unit ring carries the unit id and, in
+// Units: lane 1 of warp 3 claims them from the counter shared by all CTAs,
+// each once warp 0 has issued the previous unit's loads. A slot of the unit ring carries the unit id and, in
 // paired mode, the two union sizes and the first entries of each union, so no
 // role starts a unit with a chain of global loads.
 #include "common.cuh"
@@ -397,9 +397,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 3 && lane == 1) {
         // ================= unit claimer =================
         // Slot n of the unit ring: the unit id and, paired, its union sizes and
-        // first entries. Unit n is claimed once warp 0 has taken unit n-1, so
-        // the claim's chain of loads hides behind that unit while the dynamic
-        // longest-first order keeps a lookahead of one unit.
+        // first entries. Unit n is claimed once warp 0 has issued every load of
+        // unit n-1: the claim's chain of loads then overlaps the end of that
+        // unit, and a CTA commits to its next unit only as late as the dynamic
+        // longest-first order needs.
         bool ok = true;
         for (int n = 0; ok; ++n) {
             const int slot = n % kUnitSlots;
@@ -499,7 +500,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int i = 1; i < kUnitWords; ++i) um[i] = feed.meta(slot, i);
                     mbar_arrive(bar(L::bUEmpty + slot));
-                    if (!vrole) mbar_arrive(bar(L::bTaken));  // the claimer may take the next unit
                 }
                 const int u = um[0];
                 if (u < 0) break;
@@ -526,6 +526,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int x = 0; x < 4; ++x) cur[x] = nxt[x];
                     }
+                    // every load of this unit is issued: the claimer may take the next one
+                    if (!vrole) mbar_arrive(bar(L::bTaken));
                     continue;
                 }
                 const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
@@ -535,6 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = load_kv(cur.block(U), 0, cur.s * g.subt, U.bh);
                     cur.advance(g, U);
                 }
+                if (!vrole) mbar_arrive(bar(L::bTaken));
             }
             if (!ok) {
                 // wind down: let every copy already issued land before the CTA exits
