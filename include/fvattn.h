@@ -191,7 +191,7 @@ FVATTN_API fvattn_status fvattn_schedule(const fvattn_problem *prob, const int32
  * dense != 0 uses every block (the VSA_ALL_BLOCKS route, section 3/5), giving
  * the in-library dense comparison.
  *
- *   q, k, v        bf16 [B,H,N,D]
+ *   q, k, v        [B,H,N,D] in the problem's element type (bf16 or fp16)
  *   kv_cnt, kv_idx lists from fvattn_route (ignored if dense)
  *   work, cta_range from fvattn_schedule with the same num_ctas, dense flag
  *                  and workspace (both NULL: units in index order; with
@@ -202,7 +202,10 @@ FVATTN_API fvattn_status fvattn_schedule(const fvattn_problem *prob, const int32
  *                  r / num_ctas of list zigzag(r)), so a CTA that finishes early
  *                  takes the next unit; the last CTA resets the counter.
  *   num_ctas       grid size (0 = SM count); must match fvattn_schedule's
- *   out            bf16 [B,H,N,D]; every valid token is written
+ *   out            [B,H,N,D] in the same element type; every valid token is
+ *                  written (TMA tile stores of whole 128-byte lines), nothing
+ *                  else is touched. It must not overlap q, k or v: other CTAs
+ *                  still read those while a tile of out is stored (not checked).
  *   cta_ns         out int64 [num_ctas] busy time of each CTA in ns, or NULL
  */
 FVATTN_API fvattn_status fvattn_sparse_attn(const fvattn_problem *prob, const void *q, const void *k,
