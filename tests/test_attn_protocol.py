@@ -1,0 +1,409 @@
+"""Executable model of the attention kernel's barrier protocol (CPU).
+
+The persistent attention kernel (csrc/attn.cu) coordinates its roles only
+through mbarriers: a unit ring filled by a claimer lane, Q/K/V buffers loaded
+by TMA, S/P/O in tensor memory, and the epilogue's staged output. A protocol
+mistake there shows up on the GPU as a hang or as a buffer overwritten while
+still in use. This model replays each role's sequence of waits, arrivals,
+copies and MMA commits as in the kernel, for paired (two query tiles with
+their own key/value streams) and 128-row (both halves share each key/value
+tile) units, and runs them under random interleavings, with TMA copies
+completing in any order and each issuer's MMAs completing in issue order.
+It checks that:
+- every wait targets the phase the kernel means (its parity never aliases a
+  phase two away, in either direction) and that no run deadlocks;
+- no buffer is written while a reader still needs it and no reader sees a
+  buffer before it is filled.
+Mistakes planted in copies of the model are caught, so the checks have teeth.
+The softmax warpgroups are one agent each (their 128 arrivals count as one).
+"""
+import random
+
+import pytest
+
+SLOTS, NK, NV = 4, 2, 3
+
+
+class ProtocolError(AssertionError):
+    pass
+
+
+class Barrier:
+    def __init__(self, name, count=1):
+        self.name, self.count, self.pending, self.phase = name, count, 0, 0
+
+    def arrive(self):
+        self.pending += 1
+        if self.pending > self.count:
+            raise ProtocolError(f"{self.name}: more arrivals than its count")
+        if self.pending == self.count:
+            self.pending = 0
+            self.phase += 1
+
+    def ready(self, k):
+        """Would a parity wait for the completion of phase k return now?"""
+        if self.phase >= k + 2:
+            raise ProtocolError(f"{self.name}: wait for phase {k} lapped (now {self.phase}), parity aliases")
+        if self.phase == k - 1:
+            raise ProtocolError(f"{self.name}: wait for phase {k} would pass early on phase {k - 2}'s parity")
+        return self.phase == k + 1
+
+
+class Model:
+    def __init__(self, units, paired, mutation=None):
+        self.units = list(units)
+        self.paired = paired
+        self.mut = mutation
+        B = Barrier
+        self.b = {
+            "QFull": [B("QFull0"), B("QFull1")], "QEmpty": [B("QEmpty0"), B("QEmpty1")],
+            "KFull": [B(f"KFull{i}") for i in range(NK)], "KEmpty": [B(f"KEmpty{i}") for i in range(NK)],
+            "VFull": [B(f"VFull{i}") for i in range(NV)], "VEmpty": [B(f"VEmpty{i}") for i in range(NV)],
+            "SFull": [B("SFull0"), B("SFull1")], "SFree": B("SFree"),
+            "PFull": [B("PFull0"), B("PFull1")], "PFree": [B("PFree0"), B("PFree1")],
+            "OFull": [B("OFull0"), B("OFull1")], "OEmpty": [B("OEmpty0"), B("OEmpty1")],
+            "UFull": [B(f"UFull{i}") for i in range(SLOTS)],
+            "UEmpty": [B(f"UEmpty{i}", 6) for i in range(SLOTS)],   # producer, V, QK, PV, 2 softmax
+            "Taken": B("Taken"),
+        }
+        self.slots = [None] * SLOTS
+        self.next_unit = 0
+        # buffer states
+        self.Q = ["free", "free"]
+        self.K = ["free"] * NK
+        self.V = ["free"] * NV
+        self.S = "free"          # free -> writing -> full(h) -> free
+        self.P = ["free", "free"]
+        self.O = ["free", "free"]  # free -> acc -> complete -> free
+        self.qk_inflight = [0, 0]
+        self.async_tma = []       # (callback) completing in any order
+        self.fifo = {"qk": [], "pv": [], "st0": [], "st1": []}
+
+    # ---- helpers
+    def need(self, cond, msg):
+        if not cond:
+            raise ProtocolError(msg)
+
+    def tiles(self, u, h):
+        """Key tiles of half h: paired, its own count; otherwise the unit's
+        count for half 0 and, if the unit has a second half, for half 1."""
+        if self.paired:
+            return u[h]
+        return u[0] if (h == 0 or u[1] > 0) else 0
+
+    # ---- roles (generators yielding ("wait", barrier, phase) or ("arrive", barrier))
+    def claimer(self):
+        n = 0
+        while True:
+            if n > 0:
+                k = n - 1 if self.mut != "claim_early" else n
+                yield ("wait", self.b["Taken"], k)
+            if n >= SLOTS:
+                yield ("wait", self.b["UEmpty"][n % SLOTS], n // SLOTS - 1)
+            u = self.units[self.next_unit] if self.next_unit < len(self.units) else None
+            self.next_unit += 1
+            self.slots[n % SLOTS] = u
+            yield ("arrive", self.b["UFull"][n % SLOTS])
+            if u is None:
+                return
+            n += 1
+
+    def take(self, n):
+        slot = n % SLOTS
+        yield ("wait", self.b["UFull"][slot], n // SLOTS)
+        u = self.slots[slot]
+        yield ("arrive", self.b["UEmpty"][slot])
+        return u
+
+    def load(self, kind, idx, bar):
+        buf = getattr(self, kind)
+        self.need(buf[idx] == "free", f"{kind}[{idx}] loaded while in use ({buf[idx]})")
+        buf[idx] = "loading"
+
+        def done():
+            buf[idx] = "ready"
+            bar.arrive()
+        self.async_tma.append(done)
+
+    def producer(self):
+        kc, qloads, n = 0, [0, 0], 0
+        while True:
+            u = yield from self.take(n)
+            if u is None:
+                return
+            for h in (0, 1):
+                if self.tiles(u, h) == 0:
+                    continue
+                if qloads[h] > 0 and self.mut != "no_q_wait":
+                    yield ("wait", self.b["QEmpty"][h], qloads[h] - 1)
+                self.load("Q", h, self.b["QFull"][h])
+                qloads[h] += 1
+            nk = max(u[0], u[1]) if self.paired else u[0]
+            for r in range(nk):
+                for h in ((0, 1) if self.paired else (0,)):
+                    if self.paired and r >= u[h]:
+                        continue
+                    ks = kc % NK
+                    if kc >= NK and self.mut != "no_kempty":
+                        yield ("wait", self.b["KEmpty"][ks], kc // NK - 1)
+                    self.load("K", ks, self.b["KFull"][ks])
+                    kc += 1
+            if self.mut != "no_taken":
+                yield ("arrive", self.b["Taken"])
+            n += 1
+
+    def vproducer(self):
+        vc, n = 0, 0
+        while True:
+            u = yield from self.take(n)
+            if u is None:
+                return
+            nk = max(u[0], u[1]) if self.paired else u[0]
+            for r in range(nk):
+                for h in ((0, 1) if self.paired else (0,)):
+                    if self.paired and r >= u[h]:
+                        continue
+                    vs = vc % NV
+                    if vc >= NV:
+                        yield ("wait", self.b["VEmpty"][vs], vc // NV - 1)
+                    self.load("V", vs, self.b["VFull"][vs])
+                    vc += 1
+            n += 1
+
+    def qk_issuer(self):
+        kc, qk, qwait, n = 0, 0, [0, 0], 0
+        halves_of = lambda u: (0, 1) if (self.paired or u[1] > 0) else (0,)
+        while True:
+            u = yield from self.take(n)
+            if u is None:
+                return
+            if not self.paired:
+                for h in halves_of(u):
+                    yield ("wait", self.b["QFull"][h], qwait[h])
+                    qwait[h] += 1
+            nk = max(u[0], u[1]) if self.paired else u[0]
+            for r in range(nk):
+                hs = [h for h in (0, 1) if r < u[h]] if self.paired else list(halves_of(u))
+                if not self.paired:
+                    ks = kc % NK
+                    yield ("wait", self.b["KFull"][ks], kc // NK)
+                for h in hs:
+                    if self.paired:
+                        if r == 0:
+                            yield ("wait", self.b["QFull"][h], qwait[h])
+                            qwait[h] += 1
+                        ks = kc % NK
+                        yield ("wait", self.b["KFull"][ks], kc // NK)
+                    if qk > 0 and self.mut != "no_sfree":
+                        yield ("wait", self.b["SFree"], qk - 1)
+                    self.need(self.Q[h] == "ready", f"QK reads Q[{h}] in state {self.Q[h]}")
+                    self.need(self.K[ks] == "ready", f"QK reads K[{ks}] in state {self.K[ks]}")
+                    self.need(self.S == "free", f"QK overwrites S in state {self.S}")
+                    self.S = "writing"
+                    self.qk_inflight[h] += 1
+
+                    def qk_done(h=h):
+                        self.S = ("full", h)
+                        self.qk_inflight[h] -= 1
+                        self.b["SFull"][h].arrive()
+                    self.fifo["qk"].append(qk_done)
+                    qk += 1
+                    if self.paired:
+                        self.fifo["qk"].append(self._free_k(ks))
+                        kc += 1
+                if not self.paired:
+                    self.fifo["qk"].append(self._free_k(ks))
+                    kc += 1
+            n += 1
+
+    def _free_k(self, ks):
+        def f():
+            self.K[ks] = "free"
+            self.b["KEmpty"][ks].arrive()
+        return f
+
+    def pv_issuer(self):
+        vc, pf, oe, o_pend, n = 0, [0, 0], [0, 0], [False, False], 0
+        halves_of = lambda u: (0, 1) if (self.paired or u[1] > 0) else (0,)
+        while True:
+            u = yield from self.take(n)
+            if u is None:
+                return
+            nk = max(u[0], u[1]) if self.paired else u[0]
+            for r in range(nk):
+                hs = [h for h in (0, 1) if r < u[h]] if self.paired else list(halves_of(u))
+                if not self.paired:
+                    vs = vc % NV
+                    yield ("wait", self.b["VFull"][vs], vc // NV)
+                for h in hs:
+                    if self.paired:
+                        vs = vc % NV
+                        yield ("wait", self.b["VFull"][vs], vc // NV)
+                    yield ("wait", self.b["PFull"][h], pf[h])
+                    pf[h] += 1
+                    if r == 0 and o_pend[h] and self.mut != "no_o_free":
+                        yield ("wait", self.b["OEmpty"][h], oe[h])
+                        oe[h] += 1
+                        o_pend[h] = False
+                    self.need(self.V[vs] == "ready", f"PV reads V[{vs}] in state {self.V[vs]}")
+                    self.need(self.P[h] == "full", f"PV reads P[{h}] in state {self.P[h]}")
+                    if r == 0:
+                        self.need(self.O[h] == "free", f"PV starts O[{h}] in state {self.O[h]}")
+                        self.O[h] = "acc"
+                    last = r == (u[h] if self.paired else u[0]) - 1
+
+                    def pv_done(h=h, last=last):
+                        self.P[h] = "free"
+                        self.b["PFree"][h].arrive()
+                        if last:
+                            self.O[h] = "complete"
+                            self.b["OFull"][h].arrive()
+                    self.fifo["pv"].append(pv_done)
+                    if last:
+                        o_pend[h] = True
+                    if self.paired:
+                        self.fifo["pv"].append(self._free_v(vs))
+                        vc += 1
+                if not self.paired:
+                    self.fifo["pv"].append(self._free_v(vs))
+                    vc += 1
+            n += 1
+
+    def _free_v(self, vs):
+        def f():
+            self.V[vs] = "free"
+            self.b["VEmpty"][vs].arrive()
+        return f
+
+    def softmax(self, h):
+        sf, pw, of, n = 0, 0, 0, 0
+        while True:
+            u = yield from self.take(n)
+            n += 1
+            if u is None:
+                return
+            nt = self.tiles(u, h)
+            if nt == 0:
+                continue
+            for r in range(nt):
+                yield ("wait", self.b["SFull"][h], sf)
+                sf += 1
+                self.need(self.S == ("full", h), f"softmax {h} reads S in state {self.S}")
+                self.S = "free"
+                yield ("arrive", self.b["SFree"])
+                if pw > 0 and self.mut != "no_pfree":
+                    yield ("wait", self.b["PFree"][h], pw - 1)
+                self.need(self.P[h] == "free", f"softmax {h} overwrites P[{h}] in state {self.P[h]}")
+                self.P[h] = "full"
+                yield ("arrive", self.b["PFull"][h])
+                pw += 1
+            # epilogue: O read, staged in Q[h], stored, Q[h] handed back
+            yield ("wait", self.b["OFull"][h], of)
+            of += 1
+            self.need(self.O[h] == "complete", f"epilogue {h} reads O in state {self.O[h]}")
+            self.O[h] = "free"
+            yield ("arrive", self.b["OEmpty"][h])
+            self.need(self.Q[h] == "ready" and self.qk_inflight[h] == 0,
+                      f"epilogue {h} stages into Q[{h}] in state {self.Q[h]} with {self.qk_inflight[h]} QK in flight")
+            self.Q[h] = "staged"
+            st = self.fifo[f"st{h}"]
+
+            def read_done(h=h):
+                self.Q[h] = "stored"
+            st.append(read_done)
+            if self.mut == "early_q_release":
+                yield ("arrive", self.b["QEmpty"][h])   # before the stores have read the tile
+            yield ("drain", f"st{h}")
+            self.need(self.Q[h] == "stored", f"Q[{h}] handed back in state {self.Q[h]}")
+            self.Q[h] = "free"
+            if self.mut != "early_q_release":
+                yield ("arrive", self.b["QEmpty"][h])
+
+    # ---- scheduler
+    def run(self, rng, max_steps=200000):
+        agents = {"claimer": self.claimer(), "producer": self.producer(), "vproducer": self.vproducer(),
+                  "qk": self.qk_issuer(), "pv": self.pv_issuer(), "sm0": self.softmax(0), "sm1": self.softmax(1)}
+        pending = {name: None for name in agents}
+        done = set()
+
+        def advance(name):
+            try:
+                pending[name] = next(agents[name])
+            except StopIteration:
+                done.add(name)
+                pending[name] = None
+
+        for name in agents:
+            advance(name)
+        for _ in range(max_steps):
+            choices = []
+            for name, act in pending.items():
+                if name in done:
+                    continue
+                kind = act[0]
+                if kind == "arrive" or (kind == "wait" and act[1].ready(act[2])) or \
+                        (kind == "drain" and not self.fifo[act[1]]):
+                    choices.append(("agent", name))
+            choices += [("tma", i) for i in range(len(self.async_tma))]
+            choices += [("fifo", q) for q, items in self.fifo.items() if items]
+            if not choices:
+                if len(done) == len(agents):
+                    return
+                raise ProtocolError("deadlock: " + ", ".join(
+                    f"{n} waits on {pending[n][1].name if pending[n][0] == 'wait' else pending[n][1]}"
+                    for n in agents if n not in done))
+            kind, what = rng.choice(choices)
+            if kind == "agent":
+                act = pending[what]
+                if act[0] == "arrive":
+                    act[1].arrive()
+                advance(what)
+            elif kind == "tma":
+                self.async_tma.pop(what)()
+            else:
+                self.fifo[what].pop(0)()
+        raise ProtocolError("no progress within the step limit")
+
+
+def random_units(rng, paired, n):
+    units = []
+    for _ in range(n):
+        if paired:
+            a = rng.randint(1, 4)
+            b = rng.choice([0] + [rng.randint(1, 4)] * 5)   # an empty second tile now and then
+            units.append((a, b))
+        else:
+            units.append((rng.randint(1, 5), rng.choice([0, 1, 1, 1])))  # (key tiles, has a second half)
+    return units
+
+
+@pytest.mark.parametrize("paired", [True, False])
+def test_protocol_has_no_deadlock_or_hazard(paired):
+    rng = random.Random(1234 + paired)
+    for trial in range(150):
+        Model(random_units(rng, paired, rng.randint(1, 14)), paired).run(rng)
+
+
+@pytest.mark.parametrize("mutation", ["no_q_wait", "no_sfree", "no_pfree", "early_q_release", "no_kempty",
+                                      "claim_early", "no_taken"])
+def test_planted_protocol_mistakes_are_caught(mutation):
+    rng = random.Random(99)
+    caught = False
+    for trial in range(300):
+        try:
+            Model(random_units(rng, True, rng.randint(2, 12)), True, mutation).run(rng)
+        except ProtocolError:
+            caught = True
+            break
+    assert caught, mutation
+
+
+def test_o_free_wait_is_implied_by_p_order():
+    # The PV issuer waits for the epilogue to have read O_h before the next
+    # unit's first product into O_h. The model shows that wait never binds:
+    # that product needs P_h of the next unit, which the same softmax
+    # warpgroup writes only after its epilogue. The kernel keeps it as a guard.
+    rng = random.Random(7)
+    for trial in range(150):
+        paired = bool(trial & 1)
+        Model(random_units(rng, paired, rng.randint(1, 14)), paired, "no_o_free").run(rng)
