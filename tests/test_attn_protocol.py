@@ -17,11 +17,25 @@ It checks that:
 Mistakes planted in copies of the model are caught, so the checks have teeth.
 The softmax warpgroups are one agent each (their 128 arrivals count as one).
 """
+import os
 import random
+import re
 
 import pytest
 
-SLOTS, NK, NV = 4, 2, 3
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                   "block_sparse_attention_fvattn_b200", "csrc", "attn.cu")
+
+
+def kernel_constant(name):
+    return int(re.search(rf"constexpr int {name} = (\d+);", open(SRC).read()).group(1))
+
+
+# ring depths as the kernel declares them
+SLOTS, NK, NV = kernel_constant("kUnitSlots"), kernel_constant("kNK"), kernel_constant("kNV")
+# roles that take every unit from the ring, in warps: the Q/K and V producers,
+# the QK and PV issuers, and the 8 softmax warps
+RING_CONSUMER_WARPS = 4 + 8
 
 
 class ProtocolError(AssertionError):
@@ -407,3 +421,9 @@ def test_o_free_wait_is_implied_by_p_order():
     for trial in range(150):
         paired = bool(trial & 1)
         Model(random_units(rng, paired, rng.randint(1, 14)), paired, "no_o_free").run(rng)
+
+
+def test_unit_ring_consumer_count_matches_the_roles():
+    # the unit slots are freed after this many arrivals; each role above
+    # (a softmax warpgroup as 4 warps) arrives once per unit
+    assert kernel_constant("kUnitConsumers") == RING_CONSUMER_WARPS
