@@ -292,7 +292,11 @@ const char *fvattn_status_string(fvattn_status s)
 // fixes its device footprint at start-up. For them the routing scratch -- the
 // status word and the pooled block means of Q and K -- lives in one array
 // compiled into this library, sized kNoAllocScratchBytes. Every GPU that
-// loads the library holds that array until the process exits.
+// loads the library holds that array until the process exits. The scores are
+// always computed on the CUDA cores in fp32 here (the fixed array has no room
+// for a score matrix), so from kTcScoresMinBlocks blocks on the lists can
+// differ from fvattn_route's (which then uses the TF32 tensor-core split)
+// where two blocks' scores lie within fp32 rounding of each other.
 #include <mutex>
 
 namespace fvattn {
@@ -301,27 +305,67 @@ constexpr size_t kNoAllocScratchBytes = 16u << 20;  // 16 MiB per device
 static __device__ __align__(256) uint8_t g_route_scratch[kNoAllocScratchBytes];
 
 namespace {
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mu;
-void *g_scratch_addr[kMaxDevices];  // device address of g_route_scratch, per device, after set-up
-
 // The array's name in host code is only a stand-in for the device symbol;
-// kernels must get the device address, which is looked up once per device
-// (with that device current) and cached.
+// kernels must get its device address, which cudaGetSymbolAddress returns for
+// the context current on the calling thread. Each context (a device's primary
+// context, or a context the caller made current itself) has its own copy, so
+// the address is cached per context, keyed on the context's process-unique id
+// (cuCtxGetId): a context created later -- for example after cudaDeviceReset
+// -- gets a new id and a fresh lookup, never a stale address.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+struct ScratchEntry {
+    unsigned long long ctx_id;
+    void *addr;
+};
+constexpr int kMaxContexts = 64;
+std::mutex g_scratch_mu;
+ScratchEntry g_scratch_cache[kMaxContexts];
+int g_scratch_cached = 0;
+
+template <class Fn>
+Fn driver_fn(const char *name)
+{
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<Fn>(p);
+}
+
 cudaError_t route_scratch_address(void **out)
 {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_route_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_addr[dev] = p;
+    static CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    unsigned long long id = 0;
+    bool have_id = false;
+    CUcontext ctx = nullptr;
+    if (get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx && get_id(ctx, &id) == CUDA_SUCCESS)
+        have_id = true;
+    if (have_id) {
+        for (int i = 0; i < g_scratch_cached; ++i) {
+            if (g_scratch_cache[i].ctx_id == id) {
+                *out = g_scratch_cache[i].addr;
+                return cudaSuccess;
+            }
+        }
     }
-    *out = g_scratch_addr[dev];
+    // first call in this context (with its device current): look the array up;
+    // with lazy module loading this also loads the library's device code and
+    // maps the array
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_route_scratch);
+    if (e != cudaSuccess) return e;
+    if (!have_id && get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx &&
+        get_id(ctx, &id) == CUDA_SUCCESS)
+        have_id = true;  // the lookup above made the primary context current
+    if (have_id && g_scratch_cached < kMaxContexts) g_scratch_cache[g_scratch_cached++] = ScratchEntry{id, p};
+    *out = p;
     return cudaSuccess;
 }
 }  // namespace

@@ -221,18 +221,26 @@ FVATTN_API fvattn_status fvattn_sparse_attn(const fvattn_problem *prob, const vo
  * Some callers cannot call cudaMalloc where they route: a runtime that hands
  * a plug-in only its input and output tensors, code running under a memory
  * pool reservation that must not grow, or a process whose device footprint
- * is fixed at start-up. This entry point computes exactly what fvattn_route
- * computes, with the same arguments except the workspace: its scratch (the
- * pooled block means of Q and K) lives in a fixed 16 MiB array inside this
- * library, which every GPU that loads the library holds until the process
- * exits. The call allocates nothing (no cudaMalloc/cudaFree, no allocating
- * library routine).
+ * is fixed at start-up. This entry point computes the same routing as
+ * fvattn_route, with the same arguments except the workspace, with one
+ * difference: its block scores are always fp32 dot products on the CUDA
+ * cores, where fvattn_route scores rows of 320 or more blocks with a TF32
+ * split on the tensor cores; on such rows a block whose score lies within
+ * fp32 rounding of the boundary block's can land on the other side. Its
+ * scratch (the pooled block means of Q and K) lives in a fixed 16 MiB array
+ * inside this library, which every GPU that loads the library holds until
+ * the process exits. The call allocates nothing (no cudaMalloc/cudaFree, no
+ * allocating library routine).
  *   Limit: 4*(B*H*nb*D + B*H*D*round_up(nb,4)) plus 256 bytes must fit in
  *   16 MiB (e.g. 24 heads x 120 blocks at D=128, or 40 x 360); larger problems
  *   return FVATTN_ERR_WORKSPACE before anything is enqueued.
- *   Set-up: the first call on each device looks up the array's device address
- *   (with that device current) and caches it; make that first call before any
- *   stream capture.
+ *   Set-up: the first call in each CUDA context (normally once per device)
+ *   looks up the array's device address with that device current and caches
+ *   it per context (keyed on the context's unique id, so a context made after
+ *   cudaDeviceReset gets a fresh lookup). With lazy module loading, the CUDA
+ *   default, that first call also loads this library's device code and maps
+ *   the 16 MiB array: a caller whose device footprint must not grow later
+ *   should make one call at start-up, and before any stream capture.
  *   Sharing: every call on a device uses the same array, so calls that can
  *   overlap on the GPU (different streams, no ordering between them) race and
  *   may produce wrong lists; order them on one stream. Non-finite score rows

@@ -17,3 +17,17 @@ def pytest_configure(config):
 def oracle_lib():
     import oracle
     return oracle.get()
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Print how many routed rows each GPU parity workload matched exactly and
+    how many differed from the oracle under each excuse."""
+    try:
+        from tests import fvtest
+    except ImportError:
+        return
+    if not fvtest.RECORDED:
+        return
+    terminalreporter.write_sep("-", "routing lists vs the oracle")
+    for name, res in fvtest.RECORDED.items():
+        terminalreporter.write_line(f"{name}: {res.summary()}")

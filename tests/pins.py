@@ -207,6 +207,29 @@ def pin_sparse_attention_masked_sdpa(orc):
         np.testing.assert_allclose(out[h * N:(h + 1) * N], ref.numpy(), rtol=0, atol=1e-12)
 
 
+def pin_route_order_probs_cum(orc):
+    """The oracle's per-row outputs that the GPU checks read -- the ranking,
+    the block probabilities and the cumulative sums -- against numpy on the
+    oracle's own pooled means: order = a stable sort of the scores
+    descending (equal scores keep the lower block first: numpy's lexsort),
+    probs = the softmax of the scores in block order, cum = the running sum of
+    probs taken in that order."""
+    cases = [((12, 24, 40), (4, 8, 8), False, 0.9, 4), ((9, 20, 28), (4, 8, 8), True, 0.6, 2),
+             ((8, 12, 20), (4, 4, 4), False, 0.95, 3)]
+    for grid, block, iid, p, k_min in cases:
+        wl, g, q, k, v, qb, kb, scale, r = _route_small(orc, grid, block, p, k_min, H=2, D=32, iid=iid, seed=13)
+        s = _np_scores(qb, kb, scale)
+        P = _softmax_rows(s)
+        nb = s.shape[-1]
+        np.testing.assert_allclose(r["probs"], P, rtol=0, atol=1e-13)
+        for h in range(wl.H):
+            for i in range(nb):
+                expect = np.lexsort((np.arange(nb), -s[0, h, i]))
+                assert r["order"][0, h, i].tolist() == expect.tolist(), (grid, h, i)
+        ranked = np.take_along_axis(P, r["order"].astype(np.int64), -1)
+        np.testing.assert_allclose(r["cum"], np.cumsum(ranked, axis=-1), rtol=0, atol=1e-12)
+
+
 def pin_invariants(orc):
     grid, block = (9, 20, 28), (4, 8, 8)
     for p, k_min in [(0.9, 4), (0.5, 1), (0.97, 10)]:
@@ -308,5 +331,5 @@ def pin_fp16_inputs(orc):
 ALL_PINS = [
     pin_vsa_worked_example, pin_long_video_tokens, pin_pool_reshape_mean, pin_pool_ragged_bruteforce,
     pin_topp_bruteforce, pin_topk_reduction, pin_dense_reduction, pin_sparse_attention_masked_sdpa,
-    pin_invariants, pin_tie_order, pin_nonfinite_repair, pin_element_decode, pin_fp16_inputs,
+    pin_route_order_probs_cum, pin_invariants, pin_tie_order, pin_nonfinite_repair, pin_element_decode, pin_fp16_inputs,
 ]

@@ -120,15 +120,15 @@ def _run(wl, full_rows, dtype=torch.bfloat16):
     cnt = eng.kv_cnt.cpu().numpy()
     idx = eng.kv_idx.cpu().numpy()
 
-    # ---- routing
-    cmp = fvtest.compare_lists(cnt, idx, r, qb, kb, geo.scale, wl.p, wl.k_min)
-    assert cmp.unexcused == 0, cmp
-    assert cmp.excused_topp + cmp.excused_tie <= max(2, 0.02 * cmp.rows), cmp
+    # ---- routing: every GPU row valid, differences only under the excuses
+    bound = fvtest.score_bound(orc, g, qh, kh, qb, kb, geo.scale, tc=nb >= fvtest.TC_SCORES_MIN_BLOCKS)
+    cmp = fvtest.compare_lists(cnt, idx, r, bound, wl.p, wl.k_min)
+    fvtest.record(f"{wl.name}" + ("" if dtype == torch.bfloat16 else " fp16"), cmp)
+    assert cmp.invalid == 0, (cmp.summary(), cmp.first_invalid)
+    assert cmp.unexcused == 0, (cmp.summary(), cmp.first_unexcused)
+    assert cmp.excused_topp + cmp.excused_tie <= max(2, fvtest.EXCUSED_MAX_SHARE * cmp.rows), cmp.summary()
     probs = eng.block_probs.cpu().numpy().astype(np.float64)
     np.testing.assert_allclose(probs, r["probs"], rtol=2e-3, atol=1e-6)
-    # invariants of the GPU's own lists
-    for_rows = cnt.reshape(-1)
-    assert (for_rows >= min(wl.k_min, nb)).all() and (for_rows <= nb).all()
 
     # ---- schedule
     C = eng.num_ctas

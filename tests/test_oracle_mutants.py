@@ -39,6 +39,10 @@ MUTANTS = {
     "attn_wrong_query_block": ("const int i = token_block(g, n);", "const int i = token_block(g, 0);"),
     "f16_exponent_bias": ("else v = ldexp((double)(1024 + m), e - 25);", "else v = ldexp((double)(1024 + m), e - 24);"),
     "f16_subnormal_scale": ("if (e == 0) v = ldexp((double)m, -24);", "if (e == 0) v = ldexp((double)m, -25);"),
+    "order_store_shifted": ("if (order) order[r * (int64_t)nb + q] = rk[q].j;",
+                            "if (order) order[r * (int64_t)nb + q] = rk[q > 0 ? q - 1 : 0].j;"),
+    "probs_store_reversed": ("probs[r * (int64_t)nb + j] = P[j];", "probs[r * (int64_t)nb + j] = P[nb - 1 - j];"),
+    "probs_store_unnormalised": ("probs[r * (int64_t)nb + j] = P[j];", "probs[r * (int64_t)nb + j] = P[j] * z;"),
     "f16_inputs_read_as_bf16": ("return g->fp16 ? f16_to_f64(h) : bf16_to_f64(h);", "return bf16_to_f64(h);"),
 }
 

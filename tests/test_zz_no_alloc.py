@@ -71,6 +71,34 @@ def test_noalloc_matches_route_on_consecutive_calls():
     _same(ref_a, got4)
 
 
+def test_noalloc_long_rows_match_the_oracle():
+    # from 320 blocks on, fvattn_route scores on the tensor cores while the
+    # no-allocation path keeps fp32 CUDA-core scores; its lists are held to
+    # the parity rule against the oracle instead of bit-equality with
+    # fvattn_route, on two calls in a row
+    import math
+
+    import oracle
+    from block_sparse_attention_fvattn_b200 import fvattn as fa
+    wl = gen.WORKLOADS["wan14b_i2v_720p"]      # 40 heads x 360 blocks
+    q, k, _ = fvtest.make_on_gpu(wl)
+    got1 = _noalloc(fa, wl, q, k)
+    got2 = _noalloc(fa, wl, q, k)
+    torch.cuda.synchronize()
+    _same(got1, got2)
+    orc = oracle.get()
+    g = orc.geom(wl.B, wl.H, wl.grid, wl.block, wl.D)
+    qh, kh = q.cpu(), k.cpu()
+    qb, kb = orc.pool(g, qh), orc.pool(g, kh)
+    scale = 1.0 / math.sqrt(wl.D)
+    r = orc.route(g, qb, kb, scale, wl.p, wl.k_min)
+    bound = fvtest.score_bound(orc, g, qh, kh, qb, kb, scale, tc=False)
+    cmp = fvtest.compare_lists(got1[0].cpu().numpy(), got1[1].cpu().numpy(), r, bound, wl.p, wl.k_min)
+    assert cmp.invalid == 0 and cmp.unexcused == 0, (cmp.summary(), cmp.first_invalid, cmp.first_unexcused)
+    assert cmp.excused_topp + cmp.excused_tie <= max(2, fvtest.EXCUSED_MAX_SHARE * cmp.rows), cmp.summary()
+    np.testing.assert_allclose(got1[2].cpu().numpy(), r["probs"], rtol=2e-3, atol=1e-6)
+
+
 def test_noalloc_refuses_problems_beyond_its_array():
     from block_sparse_attention_fvattn_b200 import fvattn as fa
     wl = gen.WORKLOADS["long_393k"]          # pooled means need ~18.9 MB > 16 MiB
