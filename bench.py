@@ -5,10 +5,15 @@
 One step = one pass of the whole path over one batch of synthetic input:
 fvattn_route (block pooling, scores, Top-p + Top-k floor, repair, lists) ->
 fvattn_schedule (balanced longest-first CTA work lists) -> fvattn_sparse_attn
-(block-sparse attention over the kept blocks). Inputs are resident in HBM
-and larger than L2, so no flush is needed between steps. The default workload
-is the Wan-5B-like layer (B=1, H=24, D=128, grid 31x22x40, 4x8x8 blocks,
-p=0.9, k_min=8).
+(block-sparse attention over the kept blocks). The headline's inputs are
+resident in HBM and larger than L2, so no flush is needed between its
+steps. The default workload
+is the largest single-GPU layer, the 393k-token long video (B=1, H=12,
+D=128, grid 96x64x64, 4x8x8 blocks -> 1536 blocks, p=0.85, k_min=32); the
+other four workloads are measured after it with an L2 flush between steps and
+reported in the same line under "other_workloads". Per-kernel times are
+medians of per-step CUDA events; each workload's routing lists are checked
+against the fp64 oracle (counts of excused rows under "route_parity").
 
 The metric is attention TFLOPS on kept blocks: 4*D*sum_i |i| * sum_{j in S_i} |j|
 (valid query tokens x valid kept key tokens) divided by the step time. The
@@ -285,11 +290,39 @@ def run_reference(args, wl, world, rank):
 
 
 # ----------------------------------------------------------------------------- GPU arm
-def run_gpu(args, wl, world, rank, local):
+def l2_flusher(dev):
+    """A buffer twice the L2 size; writing it evicts the previous step's data."""
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    return torch.empty(max(2 * l2, 1 << 20), dtype=torch.uint8, device=dev)
+
+
+def route_parity(wl, q, k, cnt, idx):
+    """Routing lists of the GPU vs the fp64 oracle under the parity rule of the
+    tests (rows identical / excused at the Top-p boundary / excused as rounding
+    ties / unexcused / invalid)."""
+    import oracle
+    from tests import fvtest
+    orc = oracle.get()
+    g = orc.geom(wl.B, wl.H, wl.grid, wl.block, wl.D, fp16=q.dtype == torch.float16)
+    qh, kh = q.cpu(), k.cpu()
+    qb, kb = orc.pool(g, qh), orc.pool(g, kh)
+    scale = 1.0 / math.sqrt(wl.D)
+    r = orc.route(g, qb, kb, scale, wl.p, wl.k_min)
+    nb = cnt.shape[-1]
+    bound = fvtest.score_bound(orc, g, qh, kh, qb, kb, scale, tc=nb >= fvtest.TC_SCORES_MIN_BLOCKS)
+    res = fvtest.compare_lists(cnt, idx, r, bound, wl.p, wl.k_min)
+    return {"rows": res.rows, "identical": res.identical, "excused_topp_window": res.excused_topp,
+            "excused_rounding_tie": res.excused_tie, "unexcused": res.unexcused, "invalid": res.invalid}
+
+
+def measure(args, wl, dev, rank, world, flush, steps, warmup, pk, headline):
+    """Time route -> schedule -> attention on one workload.
+
+    Returns (fields of the JSON line, timed-region total ms, kept FLOPs per
+    step, engine, tensors). Per-kernel times are medians of per-step CUDA
+    events on the launching stream; with `flush` an L2-sized buffer is
+    written between steps (outside the events)."""
     from block_sparse_attention_fvattn_b200 import fvattn as fa
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    pk, pk_src = peaks()
     seed = wl.seed + 1000 * rank
     q, k, v = gen.make_inputs(wl, dev, seed=seed)
     edtype = torch.float16 if args.dtype == "f16" else torch.bfloat16
@@ -299,6 +332,7 @@ def run_gpu(args, wl, world, rank, local):
     geo = fa.Geometry(wl.B, wl.H, wl.D, wl.grid, wl.block, dtype=edtype)
     eng = fa.FVAttn(geo, wl.p, wl.k_min, device=dev)
     stream = torch.cuda.current_stream()
+    fl = l2_flusher(dev) if flush else None
 
     def step(evs=None):
         if evs is not None:
@@ -313,56 +347,54 @@ def run_gpu(args, wl, world, rank, local):
         if evs is not None:
             evs[3].record(stream)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
     if eng.status() != 0:
-        raise RuntimeError("device status flags raised during warm-up")
+        raise RuntimeError(f"{wl.name}: device status flags raised during warm-up")
 
-    # work done per step (lists are identical every step: same inputs)
     vs = valid_sizes(wl)
     cnt = eng.kv_cnt.cpu().numpy()
     idx = eng.kv_idx.cpu().numpy()
     F = kept_flops(wl, cnt, idx, vs)
     nb = eng.nb
     U = wl.B * wl.H * nb
-    paired = wl.block[0] * wl.block[1] * wl.block[2] == 64  # 64-token blocks run paired query tiles
-    tc_scores = nb >= 320  # the library scores rows of >= 320 blocks on the tensor cores (one more launch)
+    paired = wl.block[0] * wl.block[1] * wl.block[2] == 64
+    tc_scores = nb >= 320
     dense_F = 4 * wl.D * wl.B * wl.H * wl.N * wl.N
     route_bytes = 2 * wl.B * wl.H * wl.N * wl.D * 2 + 4 * U + 4 * int(cnt.sum())
 
-    # ---- timed region
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    clocks = ClockSampler(local)
-    clocks.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    clocks = ClockSampler(dev.index if dev.index is not None else 0) if headline else None
+    if clocks:
+        clocks.start()
     barrier(world)
     torch.cuda.synchronize()
     t_begin = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_begin.record(stream)
-    for s in range(args.steps):
+    for s in range(steps):
+        if fl is not None:
+            fl.fill_(s & 0xFF)
         step(evs[s])
     t_end.record(stream)
     torch.cuda.synchronize()
     barrier(world)
-    clk = clocks.stop()
+    clk = clocks.stop() if clocks else None
     total_ms = t_begin.elapsed_time(t_end)
-    route_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    sched_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    attn_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    total_ms_max = max_over_ranks(total_ms, world)
-    ms_per_step = total_ms_max / args.steps
-    work_all = sum_over_ranks(float(F), world)
-    value = work_all * args.steps / (total_ms_max * 1e-3) / 1e12
-    attn_avg = statistics.mean(attn_ms)
-    attn_tflops = F / (attn_avg * 1e-3) / 1e12
-    route_avg = statistics.mean(route_ms)
+    route_ms = statistics.median([e[0].elapsed_time(e[1]) for e in evs])
+    sched_ms = statistics.median([e[1].elapsed_time(e[2]) for e in evs])
+    attn_ms = statistics.median([e[2].elapsed_time(e[3]) for e in evs])
+    step_ms = statistics.median([e[0].elapsed_time(e[3]) for e in evs])
+    attn_tflops = F / (attn_ms * 1e-3) / 1e12
 
-    # ---- dense mode of the same kernel, CTA imbalance (outside the timed region)
+    # dense mode of the same kernel and the CTA imbalance (outside the timed region)
     dense_out = torch.empty_like(q)
     eng.dense(q, k, v, dense_out)
     dn = []
-    for _ in range(max(3, min(10, args.steps))):
+    for _ in range(3):
+        if fl is not None:
+            fl.fill_(1)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         eng.dense(q, k, v, dense_out)
@@ -370,6 +402,7 @@ def run_gpu(args, wl, world, rank, local):
         torch.cuda.synchronize()
         dn.append(a.elapsed_time(b))
     dense_ms = statistics.median(dn)
+    del dense_out
     eng.attend(q, k, v, out, timing=True)
     torch.cuda.synchronize()
     cta_ns = eng.cta_ns.cpu().numpy().astype(np.float64)
@@ -378,6 +411,45 @@ def run_gpu(args, wl, world, rank, local):
     imb_pred = float(cta_cost[busy].max() / cta_cost[busy].mean()) if busy.any() else 1.0
     imb_meas = float(cta_ns[busy].max() / cta_ns[busy].mean()) if busy.any() else 1.0
     status = eng.status()
+
+    hbm = pk["hbm_gbs"]
+    peak_tf = pk["bf16_tflops"]
+    fields = {
+        "workload": workload_desc(wl),
+        "value": F / (step_ms * 1e-3) / 1e12,
+        "ms_per_step": step_ms,
+        "attn_tflops_kept": attn_tflops,
+        "attn_frac_of_bf16_peak": attn_tflops / peak_tf,
+        "attn_frac_of_bf16_sustained": attn_tflops / pk.get("bf16_tflops_sustained", peak_tf),
+        "sparse_attn_ms": attn_ms, "dense_attn_ms": dense_ms, "sparse_over_dense": attn_ms / dense_ms,
+        "step_over_dense": step_ms / dense_ms, "dense_tflops": dense_F / (dense_ms * 1e-3) / 1e12,
+        "route_ms": route_ms, "route_gbs": route_bytes / (route_ms * 1e-3) / 1e9,
+        "route_frac_of_hbm": route_bytes / (route_ms * 1e-3) / 1e9 / hbm,
+        "sched_us": sched_ms * 1e3,
+        "imbalance_pred": imb_pred, "imbalance_meas": imb_meas,
+        "density_kept_flops": F / dense_F, "kept_flops_per_step": F, "device_status": status,
+        "l2": (f"{fl.numel() / 1e6:.0f} MB written between steps (outside the events)" if fl is not None else
+               f"inputs {3 * q.numel() * q.element_size() / 1e6:.0f} MB per step > L2, no flush"),
+        "steps": steps, "timing": "median of per-step CUDA events on the launching stream",
+    }
+    if rank == 0 and not args.no_parity:
+        fields["route_parity"] = route_parity(wl, q, k, cnt, idx)
+    launches = 5 + int(paired) + int(tc_scores)
+    return fields, total_ms, F, eng, (q, k, v, out), clk, launches, seed
+
+
+def run_gpu(args, wl, world, rank, local):
+    from block_sparse_attention_fvattn_b200 import fvattn as fa
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pk, pk_src = peaks()
+    stream = torch.cuda.current_stream()
+    fields, total_ms, F, eng, (q, k, v, out), clk, launches, seed = measure(
+        args, wl, dev, rank, world, flush=False, steps=args.steps, warmup=args.warmup, pk=pk, headline=True)
+    total_ms_max = max_over_ranks(total_ms, world)
+    ms_per_step = total_ms_max / args.steps
+    work_all = sum_over_ranks(float(F), world)
+    value = work_all * args.steps / (total_ms_max * 1e-3) / 1e12
 
     # ---- the same step replayed as one CUDA graph (no per-kernel events inside)
     graph_ms = None
@@ -403,24 +475,23 @@ def run_gpu(args, wl, world, rank, local):
     if not args.no_e2e:
         hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
         hout = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
-        pipe = fa.HostPipeline(geo, wl.p, wl.k_min, groups=args.e2e_groups, device=dev)
+        pipe = fa.HostPipeline(eng.geo, wl.p, wl.k_min, groups=args.e2e_groups, device=dev)
         n_e2e = max(2, min(args.steps, 10))
-
-        def e2e_step():
-            pipe(hq, hk, hv, hout)
-        e2e_step()
+        pipe(hq, hk, hv, hout)
         torch.cuda.synchronize()
         barrier(world)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(n_e2e):
-            e2e_step()
+            pipe(hq, hk, hv, hout)
         b.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(a.elapsed_time(b), world) / n_e2e
         e2e = {"value": work_all / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
-               "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": q.numel() * 2,
+               "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
+               "d2h_bytes_per_step": q.numel() * q.element_size(),
                "ms_per_step": e2e_ms, "head_groups": len(pipe.ranges)}
+        del pipe, hq, hk, hv, hout
 
     # ---- CPU oracle baseline (rank 0, N=1)
     cpu = None
@@ -428,41 +499,49 @@ def run_gpu(args, wl, world, rank, local):
         hq, hk, hv = q.cpu(), k.cpu(), v.cpu()
         val, desc, cores, _ = oracle_sample(wl, hq, hk, hv, args.cpu_budget)
         cpu = {"value": val / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+        del hq, hk, hv
+    del eng, q, k, v, out
+    torch.cuda.empty_cache()
+
+    # ---- the other workloads: compact results in the same line (rank 0 only
+    # prints; each rank measures its own replica, N=1 only by default)
+    others = {}
+    extra = [] if (args.no_extra or world > 1) else [n for n in gen.WORKLOAD_ORDER if n != wl.name]
+    for name in extra:
+        f2, _, _, e2, ts, _, _, _ = measure(args, gen.WORKLOADS[name], dev, rank, world, flush=True,
+                                            steps=min(args.steps, 10), warmup=3, pk=pk, headline=False)
+        others[name] = f2
+        del e2, ts
+        torch.cuda.empty_cache()
 
     peak_tf = pk["bf16_tflops"]
+    attn_tflops = fields["attn_tflops_kept"]
     traffic = recorded_traffic(wl.name)
+    paired = wl.block[0] * wl.block[1] * wl.block[2] == 64
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
         "config": {"workload": workload_desc(wl), "parallelism": f"replicas x{world} (heads shard, no exchange)",
-                   "l2": f"inputs {3 * q.numel() * 2 / 1e6:.0f} MB per step > L2, no flush",
-                   "seed": seed, "num_ctas": eng.num_ctas},
-        "attn_tflops_kept": attn_tflops,
-        "attn_frac_of_bf16_peak": attn_tflops / peak_tf,
-        "attn_frac_of_bf16_sustained": attn_tflops / pk.get("bf16_tflops_sustained", peak_tf),
-        "sparse_attn_ms": attn_avg, "dense_attn_ms": dense_ms, "sparse_over_dense": attn_avg / dense_ms,
-        "step_over_dense": ms_per_step / dense_ms, "dense_tflops": dense_F / (dense_ms * 1e-3) / 1e12,
-        "route_ms": route_avg, "route_gbs": route_bytes / (route_avg * 1e-3) / 1e9,
-        "route_frac_of_hbm": route_bytes / (route_avg * 1e-3) / 1e9 / pk["hbm_gbs"],
-        "sched_us": statistics.mean(sched_ms) * 1e3,
-        "imbalance_pred": imb_pred, "imbalance_meas": imb_meas,
-        "density_kept_flops": F / dense_F, "kept_flops_per_step": F, "device_status": status,
+                   "l2": fields["l2"], "seed": seed, "num_ctas": fa.default_num_ctas()},
+    }
+    line.update({k2: v2 for k2, v2 in fields.items() if k2 not in ("workload", "value", "ms_per_step", "l2",
+                                                                    "steps")})
+    line.update({
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": attn_tflops / peak_tf, "traffic": traffic,
                      "kernel": f"attn_kernel<{wl.D},128,{'paired' if paired else 'unpaired'}> (fvattn_sparse_attn)",
                      "peak_source": f"{pk_src} bf16 burst" + ("" if pk_src == "measured" else " (fallback)")
                      + (" x 1 (fp16 has the bf16 dense rate)" if args.dtype == "f16" else "")},
-        "route_roofline": {"bound": "hbm", "achieved": route_bytes / (route_avg * 1e-3) / 1e9,
-                           "peak": pk["hbm_gbs"], "unit": "GB/s",
-                           "frac": route_bytes / (route_avg * 1e-3) / 1e9 / pk["hbm_gbs"]},
+        "route_roofline": {"bound": "hbm", "achieved": fields["route_gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
+                           "frac": fields["route_frac_of_hbm"]},
         "clocks": clk,
-        # per step: pool + select (route), [pair lists +] two scheduler kernels, attention
         "graph_ms_per_step": graph_ms,
-        "gpu_launches": (5 + int(paired) + int(tc_scores)) * args.steps,
+        "gpu_launches": launches * args.steps,
         "e2e": e2e,
         "cpu_baseline": cpu,
-    }
+        "other_workloads": others or None,
+    })
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -472,7 +551,10 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="wan5b", choices=sorted(gen.WORKLOADS))
+    ap.add_argument("--workload", default="long_393k", choices=sorted(gen.WORKLOADS),
+                    help="headline workload (default: the largest, the 393k-token layer)")
+    ap.add_argument("--no-extra", action="store_true", help="skip the compact lines of the other workloads")
+    ap.add_argument("--no-parity", action="store_true", help="skip the oracle check of the routing lists")
     ap.add_argument("--impl", default="fvattn", choices=["fvattn", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle attention work")
     ap.add_argument("--no-cpu", action="store_true")
