@@ -438,6 +438,99 @@ def measure(args, wl, dev, rank, world, flush, steps, warmup, pk, headline):
     return fields, total_ms, F, eng, (q, k, v, out), clk, launches, seed
 
 
+def head_split_emulated(wl, q, k, v, dev, worlds, reps=3):
+    """The layer's heads split over W ranks emulated one after another on this
+    GPU (heads.step_emulated): the static shards, the RLB migration plan, and
+    RLB plus slack augmentation. Per mode: predicted rank loads (token pairs),
+    each rank's attention time (median of `reps` CUDA-event timings; a rank's
+    heads run alone on the whole GPU, so its time tracks its load) and their
+    max/mean, and the augmentation's additions."""
+    from block_sparse_attention_fvattn_b200 import fvattn as fa
+    from block_sparse_attention_fvattn_b200 import heads
+    H = wl.B * wl.H
+    geo1 = fa.Geometry(1, 1, wl.D, wl.grid, wl.block, dtype=q.dtype)
+    be = heads.GpuBackend(geo1, wl.p, wl.k_min, dev)
+    qf, kf, vf = (t.reshape(H, wl.N, wl.D) for t in (q, k, v))
+    stream = torch.cuda.current_stream()
+    out = {}
+    for W in worlds:
+        if W > H or W < 2:
+            continue
+        states = [heads.RankState(r, W, H, be) for r in range(W)]
+        entry = {}
+        for mode in ("static", "rlb", "rlb_sasa"):
+            for st in states:
+                st.balance = mode != "static"
+                st.sasa = mode == "rlb_sasa"
+            times = [[] for _ in range(W)]
+            plan = None
+            for rep in range(reps + 1):
+                for st in states:
+                    for name, t in (("q", qf), ("k", kf), ("v", vf)):
+                        st.buf[name][:st.S].copy_(t[st.h0:st.h1])
+                evs = {}
+
+                def timer(r, fn):
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                    fn()
+                    b.record(stream)
+                    evs[r] = (a, b)
+                plan = heads.step_emulated(states, timer)
+                torch.cuda.synchronize()
+                if rep > 0:
+                    for r, (a, b) in evs.items():
+                        times[r].append(a.elapsed_time(b))
+            ms = [statistics.median(t) for t in times]
+            loads = plan.load_after
+            e = {"rank_load_pairs": loads, "pred_imbalance": max(loads) / (sum(loads) / W),
+                 "rank_attn_ms": ms, "meas_imbalance": max(ms) / (sum(ms) / W), "critical_attn_ms": max(ms),
+                 "moves": sum(a != b for a, b in zip(plan.owner_in, plan.owner_out))}
+            if mode == "rlb_sasa":
+                e["added_pairs"] = sum(int(st.added_pairs.item()) for st in states)
+                e["added_mass"] = sum(float(st.added_mass.item()) for st in states)
+            entry[mode] = e
+        out[str(W)] = entry
+        del states
+        torch.cuda.empty_cache()
+    return out
+
+
+def head_split_distributed(args, wl, world, rank, dev):
+    """The layer's heads split over the torchrun ranks (strong scaling): every
+    rank draws the same layer, keeps its static shard and runs
+    heads.step_distributed (NCCL all-gather of the head costs, point-to-point
+    migration). Timed over the whole step, max over ranks."""
+    from block_sparse_attention_fvattn_b200 import fvattn as fa
+    from block_sparse_attention_fvattn_b200 import heads
+    H = wl.B * wl.H
+    q, k, v = gen.make_inputs(wl, dev, seed=wl.seed)
+    geo1 = fa.Geometry(1, 1, wl.D, wl.grid, wl.block, dtype=q.dtype)
+    st = heads.RankState(rank, world, H, heads.GpuBackend(geo1, wl.p, wl.k_min, dev), sasa=args.split_sasa)
+    qf, kf, vf = (t.reshape(H, wl.N, wl.D)[st.h0:st.h1] for t in (q, k, v))
+    comm = heads.TorchComm()
+    stream = torch.cuda.current_stream()
+    ms = []
+    for s in range(args.warmup + args.steps):
+        for name, t in (("q", qf), ("k", kf), ("v", vf)):
+            st.buf[name][:st.S].copy_(t)
+        barrier(world)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        heads.step_distributed(st, comm)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if s >= args.warmup:
+            ms.append(max_over_ranks(a.elapsed_time(b), world))
+    plan = st.plan
+    W = world
+    return {"world": world, "ms_per_layer": statistics.median(ms), "sasa": bool(args.split_sasa),
+            "pred_imbalance_static": max(plan.load_static) / (sum(plan.load_static) / W),
+            "pred_imbalance_rlb": max(plan.load_after) / (sum(plan.load_after) / W),
+            "moves": sum(a != b for a, b in zip(plan.owner_in, plan.owner_out))}
+
+
 def run_gpu(args, wl, world, rank, local):
     from block_sparse_attention_fvattn_b200 import fvattn as fa
     torch.cuda.set_device(local)
@@ -493,6 +586,14 @@ def run_gpu(args, wl, world, rank, local):
                "ms_per_step": e2e_ms, "head_groups": len(pipe.ranges)}
         del pipe, hq, hk, hv, hout
 
+    # ---- the layer's heads split over ranks: emulated on this GPU (N=1), or
+    # over the torchrun ranks with --split
+    split = None
+    if world == 1 and not args.no_split:
+        split = head_split_emulated(wl, q, k, v, dev, [int(x) for x in args.split_worlds.split(",") if x])
+    elif world > 1 and args.split:
+        split = head_split_distributed(args, wl, world, rank, dev)
+
     # ---- CPU oracle baseline (rank 0, N=1)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -541,6 +642,7 @@ def run_gpu(args, wl, world, rank, local):
         "e2e": e2e,
         "cpu_baseline": cpu,
         "other_workloads": others or None,
+        "head_split": split,
     })
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -555,6 +657,10 @@ def main():
                     help="headline workload (default: the largest, the 393k-token layer)")
     ap.add_argument("--no-extra", action="store_true", help="skip the compact lines of the other workloads")
     ap.add_argument("--no-parity", action="store_true", help="skip the oracle check of the routing lists")
+    ap.add_argument("--no-split", action="store_true", help="skip the emulated head split (N=1)")
+    ap.add_argument("--split-worlds", default="2,4,8", help="rank counts of the emulated head split")
+    ap.add_argument("--split", action="store_true", help="N>1: also time the head split over the ranks")
+    ap.add_argument("--split-sasa", action="store_true", help="with --split: slack augmentation on")
     ap.add_argument("--impl", default="fvattn", choices=["fvattn", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle attention work")
     ap.add_argument("--no-cpu", action="store_true")

@@ -37,6 +37,8 @@ WsLayout ws_layout(const Geo &g)
     L.head_cost = take((size_t)g.BH * sizeof(int64_t));
     L.pair_cnt = take(g.paired ? (size_t)g.BH * g.npair * sizeof(int32_t) : 0);
     L.pair_list = take(g.paired ? (size_t)g.BH * g.npair * g.nb * sizeof(int32_t) : 0);
+    L.aug_state = take(augment_state_bytes());
+    L.aug_row_tie = take((size_t)g.BH * g.nb * sizeof(long long));
     L.total = off;
     return L;
 }
@@ -251,6 +253,47 @@ fvattn_status fvattn_sparse_attn(const fvattn_problem *prob, const void *q, cons
     int kind = 0;
     if (launch_attn(g, q, k, v, kv_cnt, kv_idx, pair_cnt, pair_list, work, cta_range, num_ctas, dense ? 1 : 0, out,
                     cta_ns, status, s, &kind) != cudaSuccess)
+        return FVATTN_ERR_CUDA;
+    return FVATTN_OK;
+}
+
+fvattn_status fvattn_head_cost(const fvattn_problem *prob, const int32_t *kv_cnt, const int32_t *kv_idx,
+                               int32_t dense, int64_t *head_cost, fvattn_stream_t stream)
+{
+    Geo g;
+    fvattn_status st = resolve(prob, &g);
+    if (st != FVATTN_OK) return st;
+    if (!head_cost || (!dense && (!kv_cnt || !kv_idx))) return FVATTN_ERR_INVALID_ARG;
+    if (!aligned4(kv_cnt) || !aligned4(kv_idx) || ((uintptr_t)head_cost & 7u)) return FVATTN_ERR_INVALID_ARG;
+    if (g.BH == 0) return FVATTN_OK;
+    if (launch_head_cost(g, kv_cnt, kv_idx, dense ? 1 : 0, head_cost, (cudaStream_t)stream) != cudaSuccess)
+        return FVATTN_ERR_CUDA;
+    return FVATTN_OK;
+}
+
+fvattn_status fvattn_augment(const fvattn_problem *prob, const float *block_probs, int64_t budget, int32_t *kv_cnt,
+                             int32_t *kv_idx, int64_t *added_pairs, double *added_mass, void *ws, size_t ws_bytes,
+                             fvattn_stream_t stream)
+{
+    Geo g;
+    fvattn_status st = resolve(prob, &g);
+    if (st != FVATTN_OK) return st;
+    if (budget < 0 || !block_probs || !kv_cnt || !kv_idx) return FVATTN_ERR_INVALID_ARG;
+    if (!aligned4(block_probs) || !aligned4(kv_cnt) || !aligned4(kv_idx)) return FVATTN_ERR_INVALID_ARG;
+    if (((uintptr_t)added_pairs & 7u) || ((uintptr_t)added_mass & 7u)) return FVATTN_ERR_INVALID_ARG;
+    st = check_ws(g, ws, ws_bytes);
+    if (st != FVATTN_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (g.BH == 0) {
+        if (added_pairs && cudaMemsetAsync(added_pairs, 0, sizeof(int64_t), s) != cudaSuccess) return FVATTN_ERR_CUDA;
+        if (added_mass && cudaMemsetAsync(added_mass, 0, sizeof(double), s) != cudaSuccess) return FVATTN_ERR_CUDA;
+        return FVATTN_OK;
+    }
+    const WsLayout L = ws_layout(g);
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    if (launch_augment(g, block_probs, (long long)budget, kv_cnt, kv_idx, w + L.aug_state,
+                       reinterpret_cast<long long *>(w + L.aug_row_tie),
+                       reinterpret_cast<unsigned long long *>(added_pairs), added_mass, s) != cudaSuccess)
         return FVATTN_ERR_CUDA;
     return FVATTN_OK;
 }

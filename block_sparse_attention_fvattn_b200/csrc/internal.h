@@ -18,6 +18,8 @@ struct WsLayout {
     size_t head_cost;    // int64 [BH]         scheduler: total cost per head
     size_t pair_cnt;     // int32 [BH*npair]   paired mode: union size of each pair of query blocks
     size_t pair_list;    // int32 [BH*npair*nb] paired mode: the union, ascending, with membership flags
+    size_t aug_state;    // augmentation: radix-select state (histogram, boundary key, budget left)
+    size_t aug_row_tie;  // int64 [BH*nb]      augmentation: boundary-key cost before each row
     size_t total;
 };
 WsLayout ws_layout(const Geo &g);
@@ -53,5 +55,14 @@ cudaError_t launch_attn(const Geo &g, const void *q, const void *k, const void *
                         const int32_t *kv_idx, const int32_t *pair_cnt, const int32_t *pair_list,
                         const int32_t *work, const int32_t *cta_range, int num_ctas, int dense, void *out,
                         int64_t *cta_ns, uint32_t *status, cudaStream_t stream, int *launch_error_kind);
+
+// Work of every head (valid token pairs of its kept lists).
+cudaError_t launch_head_cost(const Geo &g, const int32_t *kv_cnt, const int32_t *kv_idx, int dense, int64_t *head_cost,
+                             cudaStream_t stream);
+// Slack augmentation of the lists (in place) within `budget` token pairs.
+cudaError_t launch_augment(const Geo &g, const float *probs, long long budget, int32_t *kv_cnt, int32_t *kv_idx,
+                           void *state, long long *row_tie, unsigned long long *added_cost, double *added_mass,
+                           cudaStream_t stream);
+size_t augment_state_bytes();
 
 }  // namespace fvattn

@@ -55,6 +55,10 @@ def _load():
         "fvattn_schedule": (i32, [P, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp]),
         "fvattn_sparse_attn": (i32, [P, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]),
         "fvattn_read_device_status": (i32, [vp, vp, ctypes.POINTER(ctypes.c_uint32)]),
+        "fvattn_head_cost": (i32, [P, vp, vp, i32, vp, vp]),
+        "fvattn_rlb_plan": (i32, [vp, i32, i32, vp, i32, vp, vp]),
+        "fvattn_lpt_assign": (i32, [vp, i32, i32, vp, vp]),
+        "fvattn_augment": (i32, [P, vp, ctypes.c_int64, vp, vp, vp, vp, vp, sz, vp]),
         "fvattn_status_string": (ctypes.c_char_p, [i32]),
     }
     for name, (res, args) in sig.items():
@@ -67,7 +71,7 @@ def _load():
 _lib = _load()
 EXPORTED = ("fvattn_num_blocks", "fvattn_default_num_ctas", "fvattn_workspace_size", "fvattn_workspace_init",
             "fvattn_route", "fvattn_route_noalloc", "fvattn_schedule", "fvattn_sparse_attn", "fvattn_read_device_status",
-            "fvattn_status_string")
+            "fvattn_status_string", "fvattn_head_cost", "fvattn_rlb_plan", "fvattn_lpt_assign", "fvattn_augment")
 
 
 def status_string(s: int) -> str:
@@ -190,6 +194,52 @@ def sparse_attn(geo: Geometry, q, k, v, kv_cnt, kv_idx, work, cta_range, num_cta
                                  _ptr(out, geo.dtype, "out"), _ptr(cta_ns, torch.int64, "cta_ns"),
                                  _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
     _check(st, "fvattn_sparse_attn")
+
+
+def head_cost(geo: Geometry, kv_cnt: Optional[torch.Tensor], kv_idx: Optional[torch.Tensor], out: torch.Tensor,
+              dense: bool = False, stream=None):
+    """out[b*H + h] (int64) = valid (query, key) token pairs of head (b, h) under its kept lists."""
+    prob = geo.problem()
+    st = _lib.fvattn_head_cost(ctypes.byref(prob), _ptr(kv_cnt, torch.int32, "kv_cnt"),
+                               _ptr(kv_idx, torch.int32, "kv_idx"), int(bool(dense)), _ptr(out, torch.int64, "out"),
+                               _stream(stream))
+    _check(st, "fvattn_head_cost")
+
+
+def rlb_plan(head_cost_host, world: int, owner_in=None, max_moves: int = 1):
+    """Head migration plan (host): returns (owner_out, rank_load) as int lists.
+    head_cost_host: sequence of int64 costs; owner_in: None for the static shards."""
+    n = len(head_cost_host)
+    costs = (ctypes.c_int64 * max(n, 1))(*[int(c) for c in head_cost_host])
+    own_in = None if owner_in is None else (ctypes.c_int32 * max(n, 1))(*[int(o) for o in owner_in])
+    own_out = (ctypes.c_int32 * max(n, 1))()
+    load = (ctypes.c_int64 * max(int(world), 1))()
+    st = _lib.fvattn_rlb_plan(costs, int(n), int(world), own_in, int(max_moves), own_out, load)
+    _check(st, "fvattn_rlb_plan")
+    return [int(own_out[h]) for h in range(n)], [int(load[r]) for r in range(int(world))]
+
+
+def lpt_assign(head_cost_host, world: int):
+    """Longest-processing-time assignment of heads to ranks (host): (owner, rank_load)."""
+    n = len(head_cost_host)
+    costs = (ctypes.c_int64 * max(n, 1))(*[int(c) for c in head_cost_host])
+    own_out = (ctypes.c_int32 * max(n, 1))()
+    load = (ctypes.c_int64 * max(int(world), 1))()
+    _check(_lib.fvattn_lpt_assign(costs, int(n), int(world), own_out, load), "fvattn_lpt_assign")
+    return [int(own_out[h]) for h in range(n)], [int(load[r]) for r in range(int(world))]
+
+
+def augment(geo: Geometry, block_probs: torch.Tensor, budget: int, kv_cnt: torch.Tensor, kv_idx: torch.Tensor,
+            ws: torch.Tensor, added_pairs: Optional[torch.Tensor] = None, added_mass: Optional[torch.Tensor] = None,
+            stream=None):
+    """Add the highest-probability unkept blocks to the lists, within `budget` token pairs (in place)."""
+    prob = geo.problem()
+    st = _lib.fvattn_augment(ctypes.byref(prob), _ptr(block_probs, torch.float32, "block_probs"), int(budget),
+                             _ptr(kv_cnt, torch.int32, "kv_cnt"), _ptr(kv_idx, torch.int32, "kv_idx"),
+                             _ptr(added_pairs, torch.int64, "added_pairs"),
+                             _ptr(added_mass, torch.float64, "added_mass"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+                             _stream(stream))
+    _check(st, "fvattn_augment")
 
 
 def read_device_status(ws: torch.Tensor, stream=None) -> int:

@@ -251,6 +251,89 @@ FVATTN_API fvattn_status fvattn_route_noalloc(const fvattn_problem *prob, const 
                                               float p, int32_t k_min, int32_t *kv_cnt, int32_t *kv_idx,
                                               float *block_probs, fvattn_stream_t stream);
 
+/*
+ * fvattn_head_cost -- the actual work of every head under its kept lists, the
+ * quantity the method's Runtime Load Balancing profiles per head before it
+ * moves heavy heads off the critical rank (ai-feeds.com FVAttn summary, "Key
+ * modules" 2; hotpaper.ai summary, RLB bullet: heads are rebalanced by their
+ * real per-head workload).
+ *
+ *   head_cost[b*H + h] = sum over query blocks i of |i| * sum_{j in S_i} |j|
+ * with |j| the valid tokens of block j: the (query, key) token pairs the
+ * attention evaluates, proportional to its FLOPs (4*D per pair). Exact int64.
+ *   kv_cnt, kv_idx  lists from fvattn_route (ignored if dense != 0: every
+ *                   block kept, cost N*N per head)
+ *   head_cost       out int64 [B*H], 8-byte aligned
+ * Asynchronous on `stream`; needs no workspace.
+ */
+FVATTN_API fvattn_status fvattn_head_cost(const fvattn_problem *prob, const int32_t *kv_cnt, const int32_t *kv_idx,
+                                          int32_t dense, int64_t *head_cost, fvattn_stream_t stream);
+
+/*
+ * fvattn_rlb_plan -- head migration plan of Runtime Load Balancing (host
+ * code; no GPU). Heads start on their owner ranks; the most loaded rank moves
+ * one of its own heads to the least loaded rank that can still receive,
+ * choosing the head that leaves the larger of the two loads smallest (ties:
+ * the heavier head, then the lower index), as long as the move shortens the
+ * critical rank; every rank sends at most max_moves heads and receives at
+ * most max_moves (the pages' setting: 1, ai-feeds.com summary "Key modules"
+ * 2: a few heavy heads move over P2P; hotpaper.ai summary: each rank sends
+ * and receives at most one head).
+ *   head_cost   host int64 [n_heads] (e.g. from fvattn_head_cost), >= 0
+ *   world       ranks (>= 1)
+ *   owner_in    host int32 [n_heads] initial owner of each head, or NULL for
+ *               the static shards: rank r holds heads [r*n/world, (r+1)*n/world)
+ *   owner_out   out host int32 [n_heads] owner after the moves
+ *   rank_load   out host int64 [world] load per rank after the moves, or NULL
+ * Deterministic: every rank computes the same plan from the same costs.
+ */
+FVATTN_API fvattn_status fvattn_rlb_plan(const int64_t *head_cost, int32_t n_heads, int32_t world,
+                                         const int32_t *owner_in, int32_t max_moves, int32_t *owner_out,
+                                         int64_t *rank_load);
+
+/*
+ * fvattn_lpt_assign -- heads to ranks from scratch by longest processing time
+ * first (host code): heads by cost descending (ties: lower index), each to the
+ * least loaded rank (ties: lower rank). For callers whose sequence-parallel
+ * all-to-all can place any head on any rank at no extra cost, so no
+ * migration limit applies; its largest load is at most (4/3 - 1/(3*world))
+ * times the best possible (Graham's bound for this rule).
+ *   head_cost  host int64 [n_heads], >= 0
+ *   owner_out  out host int32 [n_heads]
+ *   rank_load  out host int64 [world], or NULL
+ */
+FVATTN_API fvattn_status fvattn_lpt_assign(const int64_t *head_cost, int32_t n_heads, int32_t world,
+                                           int32_t *owner_out, int64_t *rank_load);
+
+/*
+ * fvattn_augment -- Slack-Aware Sparse Augmentation: spend a budget of spare
+ * work on extra high-value blocks (ai-feeds.com FVAttn summary, "Key modules"
+ * 3: ranks below the critical path insert additional attention blocks chosen
+ * by attention score without lengthening that path; hotpaper.ai summary,
+ * SASA bullet).
+ *
+ * The candidates are every (row, block j) pair of the problem whose block j
+ * the row's list does not keep; a candidate's value is its block probability
+ * P (block_probs from fvattn_route) and its cost |i| * |j| token pairs.
+ * Candidates are ordered by P descending, then row (b*H + h)*nb + i
+ * ascending, then j ascending; the longest prefix of that order whose total
+ * cost is at most `budget` is added to the lists, which stay ascending
+ * (kv_cnt grows accordingly). budget 0 changes nothing; a budget at least the
+ * cost of every candidate keeps every block.
+ *   block_probs    fp32 [B,H,nb,nb] from fvattn_route (required)
+ *   budget         token pairs, >= 0 (the rank's slack: the critical rank's
+ *                  head_cost total minus its own)
+ *   kv_cnt, kv_idx in/out, the lists of fvattn_route
+ *   added_pairs    out int64 [1] token pairs added, or NULL
+ *   added_mass     out double [1] sum of the added blocks' P, or NULL (its
+ *                  summation order is not fixed: last bits may vary)
+ *   ws, ws_bytes   the problem's workspace
+ * Asynchronous; about 11 small kernels. Run fvattn_schedule afterwards.
+ */
+FVATTN_API fvattn_status fvattn_augment(const fvattn_problem *prob, const float *block_probs, int64_t budget,
+                                        int32_t *kv_cnt, int32_t *kv_idx, int64_t *added_pairs, double *added_mass,
+                                        void *ws, size_t ws_bytes, fvattn_stream_t stream);
+
 /* Synchronise `stream`, return the device status word's flags (FVATTN_FLAG_*)
  * in *flags, and clear them. Returns CUDA on a failed copy. */
 FVATTN_API fvattn_status fvattn_read_device_status(void *ws, fvattn_stream_t stream, uint32_t *flags);

@@ -8,7 +8,7 @@ this module only compiles it with gcc and marshals numpy arrays through ctypes.
 Functions follow the steps written at the top of `fvattn_oracle.c`:
 pooling, block scores, softmax, Top-p with a Top-k floor, diagonal/non-finite
 repair, ascending kept lists, and masked softmax attention for chosen query
-tokens. Which parts are pinned to something other than the oracle itself is
+tokens; and the slack augmentation of the lists (oracle_augment). Which parts are pinned to something other than the oracle itself is
 listed in the test module `tests/test_oracle_pins.py`; the score temperature
 (scale = 1/sqrt(D) for routing) and the synthetic-input recipe are readings
 with no printed value to pin against ("parity unpinned" for those choices).
@@ -82,6 +82,7 @@ class Oracle:
         L.oracle_route.argtypes = [ctypes.POINTER(Geom), vp, vp, f64, f64, i32, vp, vp, vp, vp, vp, vp]
         L.oracle_attn_rows.argtypes = [ctypes.POINTER(Geom), vp, vp, vp, f64, vp, vp,
                                        ctypes.c_int64, vp, vp, vp, vp, vp]
+        L.oracle_augment.argtypes = [ctypes.POINTER(Geom), vp, ctypes.c_int64, vp, vp, vp, vp]
 
     @staticmethod
     def geom(B, H, grid, block, D, fp16=False) -> Geom:
@@ -128,6 +129,18 @@ class Oracle:
         self.lib.oracle_route(ctypes.byref(g), _ptr(qb), _ptr(kb), float(scale), float(p), int(k_min),
                               _ptr(cnt), _ptr(idx), _ptr(probs), _ptr(order), _ptr(cum), _ptr(nonf))
         return dict(kv_cnt=cnt, kv_idx=idx, probs=probs, order=order, cum=cum, nonfinite=nonf)
+
+    def augment(self, g: Geom, probs: np.ndarray, budget: int, kv_cnt: np.ndarray, kv_idx: np.ndarray):
+        """Slack augmentation of copies of the lists within `budget` token pairs.
+        Returns (kv_cnt, kv_idx, added_pairs, added_mass)."""
+        pr = np.ascontiguousarray(probs, dtype=np.float64)
+        cnt = np.ascontiguousarray(kv_cnt, dtype=np.int32).copy()
+        idx = np.ascontiguousarray(kv_idx, dtype=np.int32).copy()
+        pairs = ctypes.c_int64(0)
+        mass = ctypes.c_double(0.0)
+        self.lib.oracle_augment(ctypes.byref(g), _ptr(pr), ctypes.c_int64(int(budget)), _ptr(cnt), _ptr(idx),
+                                ctypes.byref(pairs), ctypes.byref(mass))
+        return cnt, idx, int(pairs.value), float(mass.value)
 
     def attn_rows(self, g: Geom, q, k, v, scale: float, rows: np.ndarray,
                   kv_cnt: Optional[np.ndarray] = None, kv_idx: Optional[np.ndarray] = None,

@@ -347,3 +347,81 @@ void oracle_attn_rows(const oracle_geom *g, const uint16_t *q, const uint16_t *k
         free(key);
     }
 }
+
+/*
+ * Slack-aware sparse augmentation (SASA) of one problem's kept lists.
+ * [ai-feeds.com FVAttn summary, "Key modules" 3: after load balancing, ranks
+ *  below the critical path spend their spare compute on extra high-value
+ *  attention blocks, chosen by attention score, without lengthening the
+ *  critical path; hotpaper.ai summary, SASA bullet.]
+ * Reading taken: a candidate is a (row, block j) pair whose block the row
+ * does not keep; its value is the block probability P[row][j] and its cost
+ * the token pairs it adds, |i| * |j|. Candidates are taken in the order of
+ * value (P descending; equal values by row, then block, ascending) for as
+ * long as the total cost stays within the budget (the rank's slack): the
+ * first candidate that does not fit ends the augmentation.
+ *   probs          [B,H,nb,nb] block probabilities (oracle_route)
+ *   kv_cnt/kv_idx  in/out: the lists, ascending
+ *   added_pairs    out: token pairs added
+ *   added_mass     out: sum of the added candidates' P
+ */
+typedef struct {
+    double p;
+    int64_t row;
+    int32_t j;
+} candidate;
+
+static int candidate_cmp(const void *a, const void *b)
+{
+    const candidate *x = (const candidate *)a, *y = (const candidate *)b;
+    if (x->p > y->p) return -1;
+    if (x->p < y->p) return 1;
+    if (x->row != y->row) return x->row < y->row ? -1 : 1;
+    return (x->j < y->j) ? -1 : (x->j > y->j);
+}
+
+void oracle_augment(const oracle_geom *g, const double *probs, int64_t budget,
+                    int32_t *kv_cnt, int32_t *kv_idx, int64_t *added_pairs, double *added_mass)
+{
+    const int nb = oracle_num_blocks(g);
+    const int64_t rows = (int64_t)g->B * g->H * nb;
+    int32_t *size = (int32_t *)malloc(sizeof(int32_t) * nb);
+    uint8_t *keep = (uint8_t *)calloc((size_t)(rows * nb), 1);
+    oracle_block_sizes(g, size);
+    for (int64_t r = 0; r < rows; ++r)
+        for (int e = 0; e < kv_cnt[r]; ++e) keep[r * nb + kv_idx[r * (int64_t)nb + e]] = 1;
+    int64_t n = 0;
+    for (int64_t x = 0; x < rows * nb; ++x) n += !keep[x];
+    candidate *c = (candidate *)malloc(sizeof(candidate) * (size_t)(n > 0 ? n : 1));
+    n = 0;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int j = 0; j < nb; ++j)
+            if (!keep[r * nb + j]) {
+                c[n].p = probs[r * (int64_t)nb + j];
+                c[n].row = r;
+                c[n].j = j;
+                ++n;
+            }
+    qsort(c, (size_t)n, sizeof(candidate), candidate_cmp);
+    int64_t spent = 0;
+    double mass = 0.0;
+    for (int64_t x = 0; x < n; ++x) {
+        const int i = (int)(c[x].row % nb);
+        const int64_t cost = (int64_t)size[i] * size[c[x].j];
+        if (spent + cost > budget) break;
+        spent += cost;
+        mass += c[x].p;
+        keep[c[x].row * nb + c[x].j] = 1;
+    }
+    for (int64_t r = 0; r < rows; ++r) {
+        int cnt = 0;
+        for (int j = 0; j < nb; ++j)
+            if (keep[r * nb + j]) kv_idx[r * (int64_t)nb + cnt++] = j;
+        kv_cnt[r] = cnt;
+    }
+    if (added_pairs) *added_pairs = spent;
+    if (added_mass) *added_mass = mass;
+    free(c);
+    free(keep);
+    free(size);
+}

@@ -293,6 +293,82 @@ def pin_nonfinite_repair(orc):
     assert (r["kv_cnt"][0, 0] < nb).any()
 
 
+# ---------------------------------------------------------------- slack augmentation
+def _augment_case(orc, grid, block, p, k_min, H=1, seed=17):
+    wl, g, q, k, v, qb, kb, scale, r = _route_small(orc, grid, block, p, k_min, H=H, D=16, iid=True, seed=seed)
+    return g, r
+
+
+def pin_augment_bruteforce_equal_costs(orc):
+    """All blocks hold 256 tokens, so every candidate costs the same: the
+    added set must have the largest mass of all candidate subsets within the
+    budget (enumerated), and never exceed it."""
+    grid, block = (8, 16, 16), (4, 8, 8)          # 8 full blocks
+    g, r = _augment_case(orc, grid, block, 0.3, 1, H=1)
+    nb = 8
+    unit = 256 * 256
+    keep = np.zeros((nb, nb), dtype=bool)
+    for i in range(nb):
+        keep[i, r["kv_idx"][0, 0, i, :r["kv_cnt"][0, 0, i]]] = True
+    cand = [(i, j) for i in range(nb) for j in range(nb) if not keep[i, j]]
+    P = r["probs"][0, 0]
+    assert len(cand) >= 8
+    for m in (0, 1, 2, 3):
+        for slack in (0, unit // 2):
+            budget = m * unit + slack
+            cnt, idx, added, mass = orc.augment(g, r["probs"], budget, r["kv_cnt"], r["kv_idx"])
+            best = max(sum(P[i, j] for i, j in comb) for comb in itertools.combinations(cand, m)) if m else 0.0
+            assert added == m * unit and added <= budget
+            assert abs(mass - best) <= 1e-12, (m, mass, best)
+            got = sum(P[i, j] for i in range(nb) for j in idx[0, 0, i, :cnt[0, 0, i]] if not keep[i, j])
+            assert abs(got - best) <= 1e-12
+            for i in range(nb):
+                lst = idx[0, 0, i, :cnt[0, 0, i]]
+                assert np.all(np.diff(lst) > 0) and set(np.flatnonzero(keep[i])) <= set(lst.tolist())
+
+
+def pin_augment_prefix_rule(orc):
+    """Ragged blocks (unequal costs): the additions are a prefix of the
+    candidates ordered by P descending (then row, then block): every added
+    candidate comes before every candidate left out, the budget holds, and
+    the first candidate left out does not fit in what remains. Budget 0
+    changes nothing; a budget covering every candidate keeps every block."""
+    grid, block = (9, 20, 28), (4, 8, 8)          # 3*3*4 = 36 blocks, ragged edges
+    g, r = _augment_case(orc, grid, block, 0.5, 2, H=2, seed=19)
+    nb = orc.num_blocks(g)
+    sizes = orc.block_sizes(g).astype(np.int64)
+    base = r["kv_cnt"].reshape(-1), r["kv_idx"].reshape(-1, nb)
+    keep = np.zeros((base[0].size, nb), dtype=bool)
+    for row in range(base[0].size):
+        keep[row, base[1][row, :base[0][row]]] = True
+    P = r["probs"].reshape(-1, nb)
+    rows, js = np.nonzero(~keep)
+    cost = sizes[rows % nb] * sizes[js]
+    order = np.lexsort((js, rows, -P[rows, js]))
+    total = int(cost.sum())
+    for budget in (0, int(cost[order[0]]) - 1, total // 7, total // 2 + 12345, total - 1, total):
+        cnt, idx, added, mass = orc.augment(g, r["probs"], budget, r["kv_cnt"], r["kv_idx"])
+        cnt, idx = cnt.reshape(-1), idx.reshape(-1, nb)
+        now = np.zeros_like(keep)
+        for row in range(cnt.size):
+            lst = idx[row, :cnt[row]]
+            assert np.all(np.diff(lst) > 0)
+            now[row, lst] = True
+        assert (now | ~keep).all(), "a kept block was dropped"
+        taken = now[rows, js][order]
+        n_taken = int(taken.sum())
+        assert taken[:n_taken].all() and not taken[n_taken:].any(), "additions are not a prefix of the order"
+        spent = int(cost[order][:n_taken].sum())
+        assert spent == added and spent <= budget
+        if n_taken < order.size:
+            assert spent + int(cost[order[n_taken]]) > budget
+        assert abs(mass - float(P[rows, js][order][:n_taken].sum())) <= 1e-12
+        if budget == 0:
+            assert n_taken == 0
+        if budget == total:
+            assert (cnt == nb).all()
+
+
 # ---------------------------------------------------------------- input types
 def pin_element_decode(orc):
     """The oracle widens every one of the 65536 bit patterns exactly like
@@ -332,4 +408,5 @@ ALL_PINS = [
     pin_vsa_worked_example, pin_long_video_tokens, pin_pool_reshape_mean, pin_pool_ragged_bruteforce,
     pin_topp_bruteforce, pin_topk_reduction, pin_dense_reduction, pin_sparse_attention_masked_sdpa,
     pin_route_order_probs_cum, pin_invariants, pin_tie_order, pin_nonfinite_repair, pin_element_decode, pin_fp16_inputs,
+    pin_augment_bruteforce_equal_costs, pin_augment_prefix_rule,
 ]

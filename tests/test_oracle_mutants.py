@@ -28,8 +28,8 @@ MUTANTS = {
     "probs_not_normalised": ("for (int j = 0; j < nb; ++j) P[j] /= z;", "(void)z;"),
     "rank_ascending": ("if (x->s > y->s) return -1;\n    if (x->s < y->s) return 1;",
                        "if (x->s < y->s) return -1;\n    if (x->s > y->s) return 1;"),
-    "tie_to_higher_index": ("return (x->j < y->j) ? -1 : (x->j > y->j);",
-                            "return (x->j > y->j) ? -1 : (x->j < y->j);"),
+    "tie_to_higher_index": ("if (x->s < y->s) return 1;\n    return (x->j < y->j) ? -1 : (x->j > y->j);",
+                            "if (x->s < y->s) return 1;\n    return (x->j > y->j) ? -1 : (x->j < y->j);"),
     "topp_count_off_by_one": ("{ m_p = q + 1; found = 1; }", "{ m_p = q; found = 1; }"),
     "floor_ignored": ("int m = m_p > k_min ? m_p : k_min;", "int m = m_p;"),
     "diagonal_not_kept": ("keep[i] = 1; /* repair", "(void)0; /* repair"),
@@ -43,6 +43,13 @@ MUTANTS = {
                             "if (order) order[r * (int64_t)nb + q] = rk[q > 0 ? q - 1 : 0].j;"),
     "probs_store_reversed": ("probs[r * (int64_t)nb + j] = P[j];", "probs[r * (int64_t)nb + j] = P[nb - 1 - j];"),
     "probs_store_unnormalised": ("probs[r * (int64_t)nb + j] = P[j];", "probs[r * (int64_t)nb + j] = P[j] * z;"),
+    "augment_ascending": ("    if (x->p > y->p) return -1;\n    if (x->p < y->p) return 1;",
+                          "    if (x->p < y->p) return -1;\n    if (x->p > y->p) return 1;"),
+    "augment_skips_and_continues": ("if (spent + cost > budget) break;", "if (spent + cost > budget) continue;"),
+    "augment_costs_query_tokens_only": ("const int64_t cost = (int64_t)size[i] * size[c[x].j];",
+                                        "const int64_t cost = (int64_t)size[i];"),
+    "augment_forgets_base_lists": ("for (int e = 0; e < kv_cnt[r]; ++e) keep[r * nb + kv_idx[r * (int64_t)nb + e]] = 1;",
+                                   "for (int e = 0; e < 0; ++e) keep[r * nb + kv_idx[r * (int64_t)nb + e]] = 1;"),
     "f16_inputs_read_as_bf16": ("return g->fp16 ? f16_to_f64(h) : bf16_to_f64(h);", "return bf16_to_f64(h);"),
 }
 
