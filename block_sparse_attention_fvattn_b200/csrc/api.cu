@@ -10,6 +10,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "fvattn.h"
 #include "internal.h"
@@ -172,11 +174,11 @@ fvattn_status fvattn_route(const fvattn_problem *prob, const void *q, const void
     cudaStream_t s = (cudaStream_t)stream;
     float *scores = g.tc_scores ? reinterpret_cast<float *>(w + L.scores) : nullptr;
     if (launch_pool(g, q, k, qbar, kbarT, s) != cudaSuccess) return FVATTN_ERR_CUDA;
-    if (scores && launch_score_gemm(g, qbar, qbar + (size_t)g.BH * g.nb * g.D, kbarT,
-                                    kbarT + (size_t)g.BH * g.nbp * g.D, scores, status, s) != cudaSuccess)
+    // the TF32 planes of each head: hi at the head's start, lo one plane later
+    if (scores && launch_score_gemm(g, qbar, qbar + (size_t)g.nb * g.D, kbarT, kbarT + (size_t)g.nbp * g.D, scores,
+                                    status, s) != cudaSuccess)
         return FVATTN_ERR_CUDA;
-    if (launch_score_select(g, qbar, kbarT, scores, p, k_min, kv_cnt, kv_idx, block_probs, status, s) !=
-        cudaSuccess)
+    if (launch_score_select(g, qbar, kbarT, scores, p, k_min, kv_cnt, kv_idx, block_probs, status, s) != cudaSuccess)
         return FVATTN_ERR_CUDA;
     return FVATTN_OK;
 }

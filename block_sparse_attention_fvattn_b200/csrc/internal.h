@@ -4,14 +4,16 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace fvattn {
 
 // Workspace carve-up (byte offsets from the workspace base; 256-byte aligned).
 struct WsLayout {
-    size_t qbar;         // fp32 [BH, nb, D]   pooled query means ([2][BH, nb, D] TF32 head, rest if tc_scores)
-    size_t kbarT;        // fp32 [BH, D, nbp]  pooled key means, transposed ([2][BH, nbp, D] if tc_scores)
+    size_t qbar;         // fp32 [BH, nb, D]   pooled query means ([BH][2][nb, D] TF32 head, rest if tc_scores)
+    size_t kbarT;        // fp32 [BH, D, nbp]  pooled key means, transposed ([BH][2][nbp, D] if tc_scores)
     size_t scores;       // fp32 [BH, nb, nbp] block scores (tc_scores only)
     size_t unit_cost;    // int32 [BH*nb]      scheduler: cost per unit
     size_t head_sorted;  // int32 [BH*nb]      scheduler: units of each head by cost
@@ -32,13 +34,16 @@ constexpr int kMaxCtas = 4096;
 cudaError_t launch_pool(const Geo &g, const void *q, const void *k, float *qbar, float *kbarT,
                         cudaStream_t stream);
 // scores != nullptr: the block scores were computed by launch_score_gemm.
+// programmatic: launched as a programmatic dependent of the kernel before it
+// on the stream (that kernel must be the one producing its inputs).
 cudaError_t launch_score_select(const Geo &g, const float *qbar, const float *kbarT, const float *scores, float p,
                                 int k_min, int32_t *kv_cnt, int32_t *kv_idx, float *probs, uint32_t *status,
-                                cudaStream_t stream);
-// Scores from means split as x = hi + lo (hi, lo exact in TF32), [BH, nb, D]
-// for Q and [BH, nbp, D] for K.
+                                cudaStream_t stream, bool programmatic = true);
+// Scores from means split as x = hi + lo (hi, lo exact in TF32), stored
+// [BH][2][nb, D] for Q and [BH][2][nbp, D] for K (hi plane, then lo plane, per
+// head): qhi/khi point at the first hi plane, qlo/klo at the first lo plane.
 cudaError_t launch_score_gemm(const Geo &g, const float *qhi, const float *qlo, const float *khi, const float *klo,
-                              float *scores, uint32_t *status, cudaStream_t stream);
+                              float *scores, uint32_t *status, cudaStream_t stream, bool programmatic = true);
 // From this many blocks on, the routing scores run on the tensor cores (at
 // 256 blocks the fused CUDA-core scoring is still faster, at 360 it is slower).
 constexpr int kTcScoresMinBlocks = 320;

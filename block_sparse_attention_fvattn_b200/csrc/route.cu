@@ -158,13 +158,14 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geo g, int nxs, cons
         const float mean = sum * (1.0f / (float)(tv * yv * (xb - xa)));
         const int j = (jt * nbh + jy) * nbw + jx0 + jl;
         if (g.tc_scores) {
-            // for the tensor cores: [2][BH, rows, D] (rows = nb for Q, nbp for
-            // K), the TF32 head of the mean and then the TF32 head of its rest
+            // for the tensor cores: [BH][2][rows, D] (rows = nb for Q, nbp for
+            // K), per head the TF32 head of the mean and then the TF32 head of
+            // its rest, so that any run of heads is one contiguous slice
             const float hi = tf32_round(mean), lo = tf32_round(mean - hi);
             const size_t rows = which ? (size_t)g.nbp : (size_t)g.nb;
             float *m = which ? kbarT : qbar;
-            m[((size_t)bh * rows + j) * D + d] = hi;
-            m[((size_t)g.BH * rows + (size_t)bh * rows + j) * D + d] = lo;
+            m[((size_t)bh * 2 * rows + j) * D + d] = hi;
+            m[((size_t)bh * 2 * rows + rows + j) * D + d] = lo;
         } else if (!which) {
             qbar[((size_t)bh * g.nb + j) * D + d] = mean;
         } else {
@@ -739,7 +740,7 @@ cudaError_t launch_pool(const Geo &g, const void *q, const void *k, float *qbar,
 template <int D, int EPL>
 static cudaError_t launch_sel_t(const Geo &g, const float *qbar, const float *kbarT, const float *scores, float p,
                                 int k_min, int32_t *kv_cnt, int32_t *kv_idx, float *probs, uint32_t *status,
-                                cudaStream_t stream)
+                                cudaStream_t stream, bool programmatic)
 {
     constexpr int ROWS = kSelRowsFor<EPL>;
     // + 32*EPL floats: a row's lanes read positions up to 32*EPL - 1
@@ -749,18 +750,23 @@ static cudaError_t launch_sel_t(const Geo &g, const float *qbar, const float *kb
     if (err != cudaSuccess) return err;
     // programmatic dependent launch: the CTAs may be scheduled while the
     // pooling kernel drains and wait in-kernel for its results
-    return launch_dependent(kern, dim3((unsigned)ceil_div(g.nb, ROWS), (unsigned)g.BH), dim3(256), smem, stream, g,
-                            qbar, kbarT, p, k_min, scores, kv_cnt, kv_idx, probs, status);
+    const dim3 grid((unsigned)ceil_div(g.nb, ROWS), (unsigned)g.BH);
+    if (programmatic)
+        return launch_dependent(kern, grid, dim3(256), smem, stream, g, qbar, kbarT, p, k_min, scores, kv_cnt, kv_idx,
+                                probs, status);
+    kern<<<grid, 256, smem, stream>>>(g, qbar, kbarT, p, k_min, scores, kv_cnt, kv_idx, probs, status);
+    return cudaGetLastError();
 }
 
 template <int D>
 static cudaError_t launch_sel_d(const Geo &g, const float *qbar, const float *kbarT, const float *scores, float p,
                                 int k_min, int32_t *kv_cnt, int32_t *kv_idx, float *probs, uint32_t *status,
-                                cudaStream_t stream)
+                                cudaStream_t stream, bool programmatic)
 {
     const int epl = ceil_div(g.nb, 32);
-#define FV_SEL(E) \
-    if (epl <= E) return launch_sel_t<D, E>(g, qbar, kbarT, scores, p, k_min, kv_cnt, kv_idx, probs, status, stream)
+#define FV_SEL(E)                                                                                                 \
+    if (epl <= E)                                                                                                 \
+    return launch_sel_t<D, E>(g, qbar, kbarT, scores, p, k_min, kv_cnt, kv_idx, probs, status, stream, programmatic)
     FV_SEL(1);
     FV_SEL(2);
     FV_SEL(4);
@@ -777,10 +783,11 @@ static cudaError_t launch_sel_d(const Geo &g, const float *qbar, const float *kb
 
 cudaError_t launch_score_select(const Geo &g, const float *qbar, const float *kbarT, const float *scores, float p,
                                 int k_min, int32_t *kv_cnt, int32_t *kv_idx, float *probs, uint32_t *status,
-                                cudaStream_t stream)
+                                cudaStream_t stream, bool programmatic)
 {
-    if (g.D == 128) return launch_sel_d<128>(g, qbar, kbarT, scores, p, k_min, kv_cnt, kv_idx, probs, status, stream);
-    return launch_sel_d<64>(g, qbar, kbarT, scores, p, k_min, kv_cnt, kv_idx, probs, status, stream);
+    if (g.D == 128)
+        return launch_sel_d<128>(g, qbar, kbarT, scores, p, k_min, kv_cnt, kv_idx, probs, status, stream, programmatic);
+    return launch_sel_d<64>(g, qbar, kbarT, scores, p, k_min, kv_cnt, kv_idx, probs, status, stream, programmatic);
 }
 
 }  // namespace fvattn

@@ -150,28 +150,31 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
         }
     } else {
         // ---- epilogue: TMEM lane = tile row; this warp owns lanes 32*(warp%4)..
+        // Each 32 x 32 chunk goes through shared memory (the operand stages
+        // are free once every MMA has completed): lane l writes its row, then
+        // the warp stores the chunk row by row, each store one contiguous
+        // 128-byte run of a score row.
         if (mbar_wait(acc_bar, 0, abort_flag)) {
             tc_fence_after();
             const int wq = warp & 3;
-            const int row = m0 + wq * 32 + lane;
-            float *srow = scores + ((size_t)bh * g.nb + row) * g.nbp;
+            float *tile = reinterpret_cast<float *>(gbase) + wq * (32 * 33);  // padded: row stride 33 floats
+            const int row0 = m0 + wq * 32;
 #pragma unroll 1
             for (int cb = 0; cb < kTileN / 32; ++cb) {
                 uint32_t r[32];
                 tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(cb * 32), r);
                 tmem_wait_ld();
                 reg_fence32(r);
-                if (row < g.nb) {
 #pragma unroll
-                    for (int q4 = 0; q4 < 8; ++q4) {
-                        const int col = n0 + cb * 32 + q4 * 4;
-                        if (col < g.nbp)
-                            *reinterpret_cast<float4 *>(srow + col) =
-                                make_float4(g.scale * __uint_as_float(r[q4 * 4]), g.scale * __uint_as_float(r[q4 * 4 + 1]),
-                                            g.scale * __uint_as_float(r[q4 * 4 + 2]),
-                                            g.scale * __uint_as_float(r[q4 * 4 + 3]));
-                    }
+                for (int c = 0; c < 32; ++c) tile[lane * 33 + c] = g.scale * __uint_as_float(r[c]);
+                __syncwarp();
+                const int col = n0 + cb * 32 + lane;
+#pragma unroll 4
+                for (int rr = 0; rr < 32; ++rr) {
+                    const int row = row0 + rr;
+                    if (row < g.nb && col < g.nbp) scores[((size_t)bh * g.nb + row) * g.nbp + col] = tile[rr * 33 + lane];
                 }
+                __syncwarp();
             }
         }
     }
@@ -205,13 +208,14 @@ static EncodeTiledFn gemm_encode_fn()
     return fn;
 }
 
-// [BH, rows, D] fp32 as a 3-D TMA tensor; box = 32 x box_rows x 1, 128-byte swizzle.
+// One plane of [BH][2][rows, D] fp32 as a 3-D TMA tensor (head stride: both
+// planes); box = 32 x box_rows x 1, 128-byte swizzle.
 static bool make_means_map(CUtensorMap *map, const Geo &g, const float *ptr, int rows, int box_rows)
 {
     EncodeTiledFn enc = gemm_encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)g.D, (cuuint64_t)rows, (cuuint64_t)g.BH};
-    const cuuint64_t strides[2] = {(cuuint64_t)g.D * 4, (cuuint64_t)rows * g.D * 4};
+    const cuuint64_t strides[2] = {(cuuint64_t)g.D * 4, (cuuint64_t)rows * g.D * 4 * 2};
     const cuuint32_t box[3] = {(cuuint32_t)kChunk, (cuuint32_t)box_rows, 1u};
     const cuuint32_t estr[3] = {1u, 1u, 1u};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(ptr), dims, strides, box, estr,
@@ -220,7 +224,7 @@ static bool make_means_map(CUtensorMap *map, const Geo &g, const float *ptr, int
 }
 
 cudaError_t launch_score_gemm(const Geo &g, const float *qhi, const float *qlo, const float *khi, const float *klo,
-                              float *scores, uint32_t *status, cudaStream_t stream)
+                              float *scores, uint32_t *status, cudaStream_t stream, bool programmatic)
 {
     CUtensorMap mqh, mql, mkh, mkl;
     if (!make_means_map(&mqh, g, qhi, g.nb, kTileM) || !make_means_map(&mql, g, qlo, g.nb, kTileM) ||
@@ -230,8 +234,11 @@ cudaError_t launch_score_gemm(const Geo &g, const float *qhi, const float *qlo, 
         cudaFuncSetAttribute(score_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (err != cudaSuccess) return err;
     const dim3 grid((unsigned)ceil_div(g.nbp, kTileN), (unsigned)ceil_div(g.nb, kTileM), (unsigned)g.BH);
-    return launch_dependent(score_gemm_kernel, grid, dim3(kGemmThreads), kSmemBytes, stream, mqh, mql, mkh, mkl, g,
-                            scores, status);
+    if (programmatic)
+        return launch_dependent(score_gemm_kernel, grid, dim3(kGemmThreads), kSmemBytes, stream, mqh, mql, mkh, mkl,
+                                g, scores, status);
+    score_gemm_kernel<<<grid, kGemmThreads, kSmemBytes, stream>>>(mqh, mql, mkh, mkl, g, scores, status);
+    return cudaGetLastError();
 }
 
 }  // namespace fvattn

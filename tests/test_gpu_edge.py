@@ -242,3 +242,38 @@ def test_exact_score_ties_follow_block_order(grid, n_k, k_min):
             if 0 < m < nb and s[0, h, i, o[m - 1]] == s[0, h, i, o[min(m, nb - 1)]]:
                 tied += 1
     assert tied >= nb // 4, tied
+
+
+def test_grouped_routing_equals_routing_the_groups_alone():
+    # a layer this large routes in head groups (selection on a side stream
+    # under the pooling of the next group); every head's lists must be the
+    # ones it gets when its half of the heads is routed as a problem of its
+    # own (small enough to route in one piece), and a CUDA-graph replay of
+    # the grouped route must give the same lists again
+    from block_sparse_attention_fvattn_b200 import fvattn as fa
+    wl = gen.custom("grouped", 1, 12, 128, (16, 64, 64), (4, 8, 8), 0.85, 8, sigma=2.0, a_range=(0.5, 4.0),
+                    seed=42)
+    q, k, v = fvtest.make_on_gpu(wl)
+    eng = _engine(wl)
+    eng.route(q, k)
+    torch.cuda.synchronize()
+    assert eng.status() == 0
+    cnt, idx = eng.kv_cnt.clone(), eng.kv_idx.clone()
+    nb = eng.nb
+    for h0, h1 in ((0, 6), (6, 12)):
+        geo = fa.Geometry(1, h1 - h0, wl.D, wl.grid, wl.block)
+        e2 = fa.FVAttn(geo, wl.p, wl.k_min)
+        e2.route(q[:, h0:h1].contiguous(), k[:, h0:h1].contiguous())
+        torch.cuda.synchronize()
+        assert torch.equal(e2.kv_cnt[0], cnt[0, h0:h1])
+        mask = torch.arange(nb, device="cuda")[None, None, :] < e2.kv_cnt[0][..., None]
+        assert torch.equal(torch.where(mask, e2.kv_idx[0], 0), torch.where(mask, idx[0, h0:h1], 0))
+    out = torch.zeros_like(q)
+    graph = eng.capture(q, k, v, out)
+    eng.kv_cnt.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(eng.kv_cnt, cnt)
+    ref = _engine(wl)(q, k, v)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)

@@ -125,7 +125,8 @@ def _worker(rank, world, port, sasa, qout):
             st.buf[name][:st.S] = t[0, st.h0:st.h1]
         heads.step_distributed(st, heads.TorchComm())
         added = int(st.added_pairs[0]) if st.added_pairs is not None else 0
-        qout.put((rank, st.output().clone(), st.plan.owner_out, st.plan.load_after, added))
+        # numpy copies pickle by value: the parent may read them after this process has exited
+        qout.put((rank, st.output().view(torch.int16).numpy().copy(), st.plan.owner_out, st.plan.load_after, added))
     finally:
         dist.destroy_process_group()
 
@@ -143,7 +144,7 @@ def test_two_gloo_ranks_match_one_process(oracle_lib, sasa):
     got = {}
     for _ in range(world):
         rank, o, owner, load, added = qout.get(timeout=300)
-        got[rank] = (o, owner, load, added)
+        got[rank] = (torch.from_numpy(o).view(torch.bfloat16), owner, load, added)
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
