@@ -3,7 +3,8 @@
 // Validation mirrors the FastVideo VSA backend's acceptance rules (zskr.cn
 // guide, section 5: bf16 tensors, equal Q/K/V head counts, no mask,
 // non-causal equal-length self-attention, a block product of 256 -- or 64 on
-// the (4,4,4) route --, grid product == sequence length; section 3: top-k
+// the (4,4,4) route; this library also takes 128 --, grid product == sequence
+// length; section 3: top-k
 // above num_blocks is rejected, top-k == num_blocks accepted). Where that
 // backend falls back to SDPA, this library returns a status instead: it has
 // no fallback path.
@@ -57,7 +58,7 @@ static fvattn_status resolve(const fvattn_problem *p, Geo *g)
     if (p->D != 64 && p->D != 128) return FVATTN_ERR_UNSUPPORTED;
     if (p->dtype != FVATTN_DTYPE_BF16 && p->dtype != FVATTN_DTYPE_F16) return FVATTN_ERR_UNSUPPORTED;
     const long long bp = (long long)p->blk_t * p->blk_h * p->blk_w;
-    if (!(bp == 256 && p->blk_t % 2 == 0) && bp != 64) return FVATTN_ERR_UNSUPPORTED;
+    if (!(bp == 256 && p->blk_t % 2 == 0) && bp != 128 && bp != 64) return FVATTN_ERR_UNSUPPORTED;
     if (p->blk_w > 256 || p->blk_h > 256 || p->blk_t > 256) return FVATTN_ERR_UNSUPPORTED;
     // the attention kernel keeps one column mask per extent along each block axis
     if (p->blk_w + p->blk_h + (bp == 256 ? p->blk_t / 2 : p->blk_t) > 40) return FVATTN_ERR_UNSUPPORTED;
@@ -84,10 +85,17 @@ static fvattn_status resolve(const fvattn_problem *p, Geo *g)
     G.BH = (int)bh;
     G.nbp = (G.nb + 3) & ~3;
     if (bp == 256) {
+        // two 128-row sub-tiles per block, the halves along t
         G.subt = G.bt / 2;
         G.nsub = 2;
         G.rows = 128;
+    } else if (bp == 128) {
+        // one 128-row sub-tile per block: one query tile per unit
+        G.subt = G.bt;
+        G.nsub = 1;
+        G.rows = 128;
     } else {
+        // 64-token blocks: two query blocks share a 128-row tile (paired)
         G.subt = G.bt;
         G.nsub = 1;
         G.rows = 64;

@@ -31,8 +31,11 @@
  *   Edge blocks hold fewer valid tokens; padded positions never act as keys
  *   and never produce output (section 6, packed [real, pad] contract).
  *   Supported: blk_t*blk_h*blk_w == 256 with blk_t even (the 256-token route,
- *   e.g. (4,8,8)) or == 64 (the 64-token (4,4,4) route, section 1), blk_w and
- *   blk_h <= 256; D in {64, 128}; nb <= 2048; B*H <= 65535.
+ *   e.g. (4,8,8)), == 64 (the 64-token (4,4,4) route, section 1), or == 128
+ *   (e.g. (2,8,8): one 128-row query tile per block, which leaves one of the
+ *   attention kernel's two softmax warpgroups idle -- correct, about half the
+ *   throughput of the other routes); blk_w + blk_h + (blk_t, or blk_t/2 for
+ *   256-token blocks) <= 40; D in {64, 128}; nb <= 2048; B*H <= 65535.
  * Pointers.  Device pointers unless stated; 16-byte aligned. The caller owns
  *   every buffer. The library allocates no device memory; the only state it
  *   keeps is per-device function attributes and a cached driver entry point.

@@ -39,6 +39,13 @@ def test_every_declared_symbol_is_exported(fa):
     assert set(declared_functions()) <= set(fa.EXPORTED) | set(declared_functions())
 
 
+def test_128_token_blocks_accepted(fa):
+    # (2,8,8): one 128-row query tile per block
+    g = fa.Geometry(1, 2, 128, (7, 20, 28), (2, 8, 8))
+    assert fa.num_blocks(g) == 4 * 3 * 4
+    assert fa.workspace_size(g) > 0
+
+
 def test_num_blocks_worked_example(fa):
     # zskr.cn VSA guide, section 3: (31,22,40) with (4,8,8) -> 8*3*5 = 120 blocks
     g = fa.Geometry(1, 24, 128, (31, 22, 40), (4, 8, 8))
@@ -50,7 +57,8 @@ def test_num_blocks_worked_example(fa):
 
 @pytest.mark.parametrize("geo_args,expect", [
     (dict(B=1, H=1, D=96, grid=(8, 16, 16), block=(4, 8, 8)), "UNSUPPORTED"),      # head dim
-    (dict(B=1, H=1, D=128, grid=(8, 16, 16), block=(2, 8, 8)), "UNSUPPORTED"),     # 128-token blocks
+    (dict(B=1, H=1, D=128, grid=(8, 16, 16), block=(3, 8, 8)), "UNSUPPORTED"),     # 192-token blocks
+    (dict(B=1, H=1, D=128, grid=(8, 16, 16), block=(2, 4, 4)), "UNSUPPORTED"),     # 32-token blocks
     (dict(B=1, H=1, D=128, grid=(8, 16, 16), block=(1, 16, 16)), "UNSUPPORTED"),   # odd blk_t, 256 tokens
     (dict(B=1, H=1, D=128, grid=(0, 16, 16), block=(4, 8, 8)), "INVALID_ARG"),     # empty grid axis
     (dict(B=1, H=1, D=128, grid=(8, 16, 16), block=(0, 8, 8)), "INVALID_ARG"),

@@ -65,7 +65,7 @@ def test_outputs_write_nothing_outside_their_extent(wl):
     nb = fa.num_blocks(geo)
     C = 148
     BH = wl.B * wl.H
-    units = nb if wl.block[0] * wl.block[1] * wl.block[2] == 256 else -(-nb // 4)
+    units = -(-nb // 4) if wl.block[0] * wl.block[1] * wl.block[2] == 64 else nb
     ws = torch.zeros(fa.workspace_size(geo, C), dtype=torch.uint8, device="cuda")
     fa.workspace_init(ws)
     s16 = _signed(SENT_16, 16)

@@ -30,6 +30,9 @@ SMALL = [
     # 15 64-token blocks: the last pair holds one query block, the last unit one and a half pairs
     gen.custom("blk64_odd_pairs", 2, 2, 128, (4, 12, 20), (4, 4, 4), 0.8, 2, sigma=1.5, a_range=(0.5, 4.0),
                seed=27),
+    # 128-token (2,8,8) blocks, ragged along every axis: one 128-row query tile per unit
+    gen.custom("blk128_ragged", 1, 3, 128, (7, 20, 28), (2, 8, 8), 0.9, 3, sigma=2.0, a_range=(0.5, 4.0), seed=28),
+    gen.custom("blk128_d64", 2, 2, 64, (8, 16, 24), (2, 8, 8), 0.85, 2, sigma=1.5, a_range=(0.5, 3.0), seed=29),
 ]
 FULL = [gen.WORKLOADS[n] for n in gen.WORKLOAD_ORDER]
 
@@ -42,8 +45,9 @@ def _oracle_route(orc, wl, q, k):
 
 
 def _units_per_head(wl, nb):
+    """64-token blocks run four query blocks per unit; the other routes one."""
     bt, bh, bw = wl.block
-    return nb if bt * bh * bw == 256 else -(-nb // 4)
+    return -(-nb // 4) if bt * bh * bw == 64 else nb
 
 
 def _host_costs(wl, nb, kv_cnt, kv_idx):
@@ -166,7 +170,7 @@ def test_small_every_row(wl):
     _run(wl, full_rows=True)
 
 
-@pytest.mark.parametrize("name", ["ragged_256tok", "blk64", "blk64_ragged_d64"])
+@pytest.mark.parametrize("name", ["ragged_256tok", "blk64", "blk64_ragged_d64", "blk128_ragged"])
 def test_small_fp16_every_row(name):
     # fp16 Q, K, V: the same path with fp16 TMA tiles, fp16 MMAs and fp16 P and O
     _run([w for w in SMALL if w.name == name][0], full_rows=True, dtype=torch.float16)
