@@ -35,8 +35,9 @@ WsLayout ws_layout(const Geo &g)
     L.qbar = take(planes * g.BH * g.nb * g.D * sizeof(float));
     L.kbarT = take(planes * g.BH * g.D * g.nbp * sizeof(float));
     L.scores = take(g.tc_scores ? (size_t)g.BH * g.nb * g.nbp * sizeof(float) : 0);
-    L.unit_cost = take((size_t)g.BH * g.nb * sizeof(int32_t));
-    L.head_sorted = take((size_t)g.BH * g.nb * sizeof(int32_t));
+    L.unit_cost = take((size_t)g.BH * (g.nb + g.npair) * sizeof(int32_t));
+    L.head_sorted = take((size_t)g.BH * (g.nb + 2) * sizeof(int32_t));
+    L.head_len = take((size_t)g.BH * sizeof(int32_t));
     L.head_cost = take((size_t)g.BH * sizeof(int64_t));
     L.pair_cnt = take(g.paired ? (size_t)g.BH * g.npair * sizeof(int32_t) : 0);
     L.pair_list = take(g.paired ? (size_t)g.BH * g.npair * g.nb * sizeof(int32_t) : 0);
@@ -226,7 +227,8 @@ fvattn_status fvattn_schedule(const fvattn_problem *prob, const int32_t *kv_cnt,
         return FVATTN_ERR_CUDA;
     if (launch_schedule(g, kv_cnt, kv_idx, dense ? 1 : 0, num_ctas, work, cta_range, cta_cost,
                         reinterpret_cast<int32_t *>(w + L.unit_cost), reinterpret_cast<int32_t *>(w + L.head_sorted),
-                        reinterpret_cast<int64_t *>(w + L.head_cost), pair_cnt, s) != cudaSuccess)
+                        reinterpret_cast<int32_t *>(w + L.head_len), reinterpret_cast<int64_t *>(w + L.head_cost),
+                        pair_cnt, s) != cudaSuccess)
         return FVATTN_ERR_CUDA;
     return FVATTN_OK;
 }

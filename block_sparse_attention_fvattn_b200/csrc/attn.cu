@@ -116,12 +116,14 @@ struct AttnLayout {
                          bVEmpty = bVFull + kNV, bSFull = bVEmpty + kNV, bSFree = bSFull + 2, bPFull = bSFree + 1,
                          bPFree = bPFull + 2, bOFull = bPFree + 2, bOEmpty = bOFull + 2, bDrain = bOEmpty + 2,
                          bUFull = bDrain + 2, bUEmpty = bUFull + kUnitSlots, bOStaged = bUEmpty + kUnitSlots,
-                         bTaken = bOStaged + 2, kNumBars = bTaken + 1;
+                         bTaken = bOStaged + 2, bComb = bTaken + 1, kNumBars = bComb + 1;
     // arrivals that free a unit slot: the two producers, the QK and PV issuers
     // and the 8 softmax warps
     static constexpr int kUnitConsumers = 12;
     static constexpr int kMisc = kBar + kNumBars * 8;
-    static constexpr int kBytes = kMisc + 64;
+    // split units (paired): the second half's row maximum and sum, per row
+    static constexpr int kComb = kMisc + 64;
+    static constexpr int kBytes = kComb + (PAIRED ? 128 * 8 : 0);
     static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
     static_assert(kAlloc <= 227 * 1024, "shared memory per CTA");
     // TMEM columns
@@ -188,22 +190,53 @@ struct TileCursor {
 
 // Paired mode: unit u = query blocks 4q .. 4q+3 of head bh; tile half h runs
 // pair 2q+h, i.e. query blocks 4q+2h (rows 0-63) and 4q+2h+1 (rows 64-127).
+// A split unit (id BH*upb + bh*npair + p, from the scheduler) runs one pair p
+// on both halves: the same query rows, half 0 over the first ceil(tiles/2)
+// tiles of the pair's union and half 1 over the rest; half 0 combines the two
+// partial results and stores the tile.
 struct PairUnit {
     int bh, q;
-    int c0, c1;                  // union size of each half's pair (0: no query block)
-    const int32_t *l0, *l1;      // the unions; nullptr in dense mode (entry e = block e, kept by both)
+    int p0, p1;                  // pair of each half
+    int split;                   // 1: one pair over both halves
+    int c0, c1;                  // union entries of each half (0: nothing)
+    const int32_t *l0, *l1;      // the entries; nullptr in dense mode (entry e = block e, kept by both)
     // per-half accessors (selects, so that the struct stays in registers)
     __device__ __forceinline__ int cnt(int h) const { return h ? c1 : c0; }
     __device__ __forceinline__ int tiles(int h) const { return (cnt(h) + 1) >> 1; }
     __device__ __forceinline__ const int32_t *list(int h) const { return h ? l1 : l0; }
+    __device__ __forceinline__ int pair(int h) const { return h ? p1 : p0; }
 };
+
+// Entries of a split pair's union that half 0 takes: its first ceil(tiles/2) tiles.
+__device__ __forceinline__ int split_first(int c)
+{
+    const int tiles = (c + 1) >> 1;
+    return min(c, 2 * ((tiles + 1) >> 1));
+}
 
 __device__ __forceinline__ PairUnit load_pair_unit(const Geo &g, int u, const int32_t *pair_cnt,
                                                    const int32_t *pair_list, int dense)
 {
     PairUnit P;
+    const int n_plain = g.BH * g.upb;
+    if (u >= n_plain) {
+        const int idx = u - n_plain;
+        P.bh = idx / g.npair;
+        P.p0 = P.p1 = idx - P.bh * g.npair;
+        P.q = P.p0 >> 1;
+        P.split = 1;
+        const int c = __ldg(pair_cnt + idx);
+        P.c0 = split_first(c);
+        P.c1 = c - P.c0;
+        P.l0 = pair_list + (size_t)idx * g.nb;
+        P.l1 = P.c1 > 0 ? P.l0 + P.c0 : nullptr;
+        return P;
+    }
     P.bh = u / g.upb;
     P.q = u - P.bh * g.upb;
+    P.p0 = 2 * P.q;
+    P.p1 = 2 * P.q + 1;
+    P.split = 0;
     P.c0 = P.c1 = 0;
     P.l0 = P.l1 = nullptr;
     for (int h = 0; h < 2; ++h) {
@@ -230,15 +263,29 @@ __device__ __forceinline__ PairUnit load_pair_unit(const Geo &g, int u, const in
     return P;
 }
 
-// The same from the union sizes published in the unit ring (no loads).
+// The same from the entry counts published in the unit ring (no loads).
 __device__ __forceinline__ PairUnit pair_unit_from(const Geo &g, int u, int c0, int c1, const int32_t *pair_list,
                                                    int dense)
 {
     PairUnit P;
-    P.bh = u / g.upb;
-    P.q = u - P.bh * g.upb;
+    const int n_plain = g.BH * g.upb;
     P.c0 = c0;
     P.c1 = c1;
+    if (u >= n_plain) {
+        const int idx = u - n_plain;
+        P.bh = idx / g.npair;
+        P.p0 = P.p1 = idx - P.bh * g.npair;
+        P.q = P.p0 >> 1;
+        P.split = 1;
+        P.l0 = pair_list + (size_t)idx * g.nb;
+        P.l1 = c1 > 0 ? P.l0 + c0 : nullptr;
+        return P;
+    }
+    P.bh = u / g.upb;
+    P.q = u - P.bh * g.upb;
+    P.p0 = 2 * P.q;
+    P.p1 = 2 * P.q + 1;
+    P.split = 0;
     const size_t pid = (size_t)P.bh * g.npair + 2 * P.q;
     P.l0 = (dense || c0 == 0) ? nullptr : pair_list + pid * g.nb;
     P.l1 = (dense || c1 == 0) ? nullptr : pair_list + (pid + 1) * g.nb;
@@ -361,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int b = 0; b < L::kNumBars; ++b) {
             uint32_t cnt = 1;
             if (b == L::bSFree || b == L::bPFull || b == L::bPFull + 1 || b == L::bOEmpty || b == L::bOEmpty + 1 ||
-                b == L::bOStaged || b == L::bOStaged + 1)
+                b == L::bOStaged || b == L::bOStaged + 1 || b == L::bComb)
                 cnt = 128;  // arrived on by all 128 threads of a softmax warpgroup
             if (b >= L::bUEmpty && b < L::bUEmpty + kUnitSlots) cnt = L::kUnitConsumers;
             mbar_init(bar(b), cnt);
@@ -384,7 +431,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Units are taken dynamically, longest first, from a counter shared by all
     // CTAs (workspace header word 1); the producer thread takes them and hands
     // them to the other roles through the unit ring.
-    const long long n_units = (long long)g.BH * g.upb;
+    // ranks to take: the scheduler's unit count (paired layers split long
+    // units), or every unit in index order without a schedule; a count beyond
+    // what any schedule can hold is refused
+    const long long n_max = (long long)g.BH * (g.upb + (PAIRED ? g.npair : 0));
+    long long n_units = work ? (long long)__ldg(cta_range + gridDim.x) : (long long)g.BH * g.upb;
+    if (n_units < 0 || n_units > n_max) {
+        if (threadIdx.x == 0) atomicOr(status, kFlagBadWork);
+        n_units = 0;
+    }
     uint32_t *unit_cursor = status + 1, *ctas_done = status + 2;
     volatile int32_t *unit_slots = reinterpret_cast<volatile int32_t *>(gbase + L::kUnit);
     UnitFeed feed{bar(L::bUFull), unit_slots, 0};
@@ -409,13 +464,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 !mbar_wait(bar(L::bUEmpty + slot), (uint32_t)((n / kUnitSlots) - 1) & 1u, abort_flag))
                 break;
             const long long r = (long long)atomicAdd(unit_cursor, 1u);
-            const int u = r < n_units ? rank_to_unit(r, work, cta_range) : -1;
+            int u = r < n_units ? rank_to_unit(r, work, cta_range) : -1;
+            // a unit id out of range, or a CTA busy far beyond any real layer
+            // (20 s), ends this CTA's units with a flag instead of running on
+            if (u >= n_max || u < -1 || globaltimer_ns() - t_start > 20000000000ull) {
+                atomicOr(status, kFlagBadWork);
+                u = -1;
+            }
             int m[kUnitWords];
             m[0] = u;
 #pragma unroll
             for (int i = 1; i < kUnitWords; ++i) m[i] = 0;
             if (PAIRED && u >= 0) {
-                const PairUnit P = load_pair_unit(g, u, pair_cnt, pair_list, dense);
+                PairUnit P = load_pair_unit(g, u, pair_cnt, pair_list, dense);
+                if (P.c0 < 0 || P.c1 < 0 || P.c0 > g.nb || P.c1 > g.nb || (P.split && P.c0 + P.c1 > g.nb)) {
+                    atomicOr(status, kFlagBadWork);
+                    P.c0 = P.c1 = 0;
+                }
                 m[1] = P.c0;
                 m[2] = P.c1;
                 m[3] = pair_entry(P.l0, P.c0, 0);
@@ -507,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const PairUnit P = pair_unit_from(g, u, um[1], um[2], pair_list, dense);
                     for (int h = 0; h < 2 && ok && !vrole; ++h) {
                         if (P.cnt(h) == 0) continue;
-                        const int qa = 2 * (2 * P.q + h);  // rows 0-63: block qa, rows 64-127: block qa+1
+                        const int qa = 2 * P.pair(h);  // rows 0-63: block qa, rows 64-127: block qa+1
                         ok = load_q(h, qa, qa + 1 < g.nb ? 2 : 1, 0, P.bh);
                     }
                     // key/value tiles, the two halves interleaved: round r is tile r of
@@ -743,7 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the key block there was kept by this row's query block); apply_mask
         // masks padding inside kept columns.
         auto tile = [&](bool first, uint32_t keep, auto &&apply_mask) -> bool {
-            if (!mbar_wait(bar(L::bSFull + h), sf & 1, abort_flag)) return false;
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar(L::bSFull + h), sf & 1, abort_flag))) return false;
             ++sf;
             tc_fence_after();
             // all BKV columns in one batch, one wait; the register fences keep
@@ -824,7 +889,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 sum = t0 + t1;
             }
             // P_h and O_h are free once the PV of this half's previous sub-tile is done
-            if (pw > 0 && !mbar_wait(bar(L::bPFree + h), (pw - 1) & 1, abort_flag)) return false;
+            if (pw > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(bar(L::bPFree + h), (pw - 1) & 1, abort_flag)))
+                return false;
             tc_fence_after();
 #pragma unroll
             for (int c = 0; c < BKV / 32; ++c) tmem_st16(tP + c * 16, pk + c * 16);
@@ -854,28 +920,65 @@ __global__ void __launch_bounds__(kThreads, 1)
         // outside the grid; the Q tile goes back to the producer once the stores
         // have read it
         const uint32_t o_stage = sbase + L::kQ + (uint32_t)(h * L::kDH * L::kQSlab) + (uint32_t)row * 128u;
-        auto epilogue = [&](int ubh, int i0, int nblk, int t_off) -> bool {
-            if (!mbar_wait(bar(L::bOFull + h), of & 1, abort_flag)) return false;
+        // split units: the second half's row maximum and sum
+        float2 *comb = reinterpret_cast<float2 *>(gbase + L::kComb);
+        int of1 = 0, cb = 0;  // half 0: phases of O_1's completion seen so far, split units combined
+        int st = 0;           // epilogues of this half that staged a tile (the storing thread's phases)
+        // comb_in (half 0 of a split unit): O = (O_0 2^(m0-m) + O_1 2^(m1-m)) / (l0 2^(m0-m) + l1 2^(m1-m)),
+        // m = max(m0, m1), with (m1, l1) published by half 1 and O_1 read from TMEM
+        auto epilogue = [&](int ubh, int i0, int nblk, int t_off, bool comb_in, int of1_phase) -> bool {
+            // every wait's outcome is agreed by the whole warp before the next
+            // warp-collective TMEM access or the caller's loop exit
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar(L::bOFull + h), of & 1, abort_flag))) return false;
             ++of;
+            float w0, w1 = 0.f;
+            if (comb_in) {
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar(L::bOFull + 1), of1_phase & 1, abort_flag))) return false;
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar(L::bComb), cb & 1, abort_flag))) return false;
+                ++cb;
+                const float2 c1 = comb[row];
+                // every real row keeps a block in one half at least; padded rows are never stored
+                const float mm = fmaxf(m, c1.x);
+                const float a0 = m == -INFINITY ? 0.f : ex2_approx(m - mm);
+                const float a1 = c1.x == -INFINITY ? 0.f : ex2_approx(c1.x - mm);
+                const float inv = 1.0f / (l * a0 + c1.y * a1);
+                w0 = a0 * inv;
+                w1 = a1 * inv;
+            } else {
+                w0 = 1.0f / l;
+            }
             tc_fence_after();
-            const float inv = 1.0f / l;
+            const uint32_t tO1 = tmem + t_lane + L::tm_o(1);
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
                 tmem_ld32(tO + c * 32, o);
-                tmem_wait_ld();
+                if (comb_in) {
+                    uint32_t o1[32];
+                    tmem_ld32(tO1 + c * 32, o1);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int v = 0; v < 32; ++v)
+                        o[v] = __float_as_uint(__uint_as_float(o[v]) * w0 + __uint_as_float(o1[v]) * w1);
+                } else {
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int v = 0; v < 32; ++v) o[v] = __float_as_uint(__uint_as_float(o[v]) * w0);
+                }
                 if (c == D / 32 - 1) {
-                    // O_h has been read: the next unit's first product may overwrite it
+                    // O_h (and, combining, O_1) have been read: the next unit's
+                    // first product may overwrite them
                     tc_fence_before();
                     mbar_arrive(bar(L::bOEmpty + h));
+                    if (comb_in) mbar_arrive(bar(L::bOEmpty + 1));
                 }
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
                     uint4 w;
-                    w.x = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 0]) * inv, __uint_as_float(o[q4 * 8 + 1]) * inv);
-                    w.y = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 2]) * inv, __uint_as_float(o[q4 * 8 + 3]) * inv);
-                    w.z = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 4]) * inv, __uint_as_float(o[q4 * 8 + 5]) * inv);
-                    w.w = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 6]) * inv, __uint_as_float(o[q4 * 8 + 7]) * inv);
+                    w.x = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 0]), __uint_as_float(o[q4 * 8 + 1]));
+                    w.y = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 2]), __uint_as_float(o[q4 * 8 + 3]));
+                    w.z = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 4]), __uint_as_float(o[q4 * 8 + 5]));
+                    w.w = pack16x2<F16>(__uint_as_float(o[q4 * 8 + 6]), __uint_as_float(o[q4 * 8 + 7]));
                     // 16-byte piece j of the row: slab j / 8, 128-byte swizzle of piece j % 8
                     const int j = c * 4 + q4;
                     st_shared_v4(o_stage + (uint32_t)((j >> 3) * L::kQSlab) + (uint32_t)(((j & 7) ^ (row & 7)) << 4),
@@ -886,8 +989,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             // storing thread waits (with the usual time limit) for all 128 rows
             fence_proxy_async();
             mbar_arrive(bar(L::bOStaged + h));
+            // phase of this staging: staged epilogues so far (a split unit's second
+            // half completes O_1 without staging)
+            const int st_phase = st++;
+            bool stored = true;
             if (row == 0) {
-                if (!mbar_wait(bar(L::bOStaged + h), (of - 1) & 1, abort_flag)) return false;
+                stored = mbar_wait(bar(L::bOStaged + h), st_phase & 1, abort_flag);
+            }
+            if (row == 0 && stored) {
                 for (int s2 = 0; s2 < nblk; ++s2) {
                     int jt, jy, jx;
                     block_coords(g, i0 + s2, jt, jy, jx);
@@ -899,11 +1008,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bulk_wait_read_all();
                 mbar_arrive(bar(L::bQEmpty + h));
             }
-            return true;
+            // the storing thread's outcome, agreed by its warp
+            return __all_sync(0xFFFFFFFFu, stored);
         };
         while (ok) {
             int slot;
             const int u = feed.next(abort_flag, ok, slot);
+            ok = __all_sync(0xFFFFFFFFu, ok);  // the warp leaves the loop together, or not at all
             if (!ok) break;
             int mc0 = 0, mc1 = 0, me0 = 0, me1 = 0;
             if constexpr (PAIRED) {
@@ -919,6 +1030,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const PairUnit P = pair_unit_from(g, u, mc0, mc1, pair_list, dense);
                 const int c_h = P.cnt(h), n_h = P.tiles(h);
                 const int32_t *lst = P.list(h);
+                // phases of O_1's completion: one per unit in which half 1 has tiles
+                const int of1_phase = of1;
+                if (P.tiles(1) > 0) ++of1;
                 if (n_h == 0) continue;
                 const int hb = row >> 6;                   // 0: first query block of the pair, 1: second
                 const int keeper = hb ? kPairInB : kPairInA;
@@ -965,8 +1079,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ent1 = nxt1;
                 }
                 if (!ok) break;
-                const int qa = 2 * (2 * P.q + h);
-                if (!epilogue(P.bh, qa, qa + 1 < g.nb ? 2 : 1, 0)) { ok = false; break; }
+                if (P.split && h == 1) {
+                    // second half of a split unit: once O_1 is complete, publish
+                    // the row maximum and sum and hand Q_1 back (its products are
+                    // done); half 0 reads O_1, combines and stores the tile
+                    if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar(L::bOFull + 1), of & 1, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    ++of;
+                    comb[row] = make_float2(m, l);
+                    mbar_arrive(bar(L::bComb));
+                    if (row == 0) mbar_arrive(bar(L::bQEmpty + 1));
+                    continue;
+                }
+                const int qa = 2 * P.pair(h);
+                if (!epilogue(P.bh, qa, qa + 1 < g.nb ? 2 : 1, 0, P.split && P.tiles(1) > 0, of1_phase)) {
+                    ok = false;
+                    break;
+                }
                 continue;
             }
             const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
@@ -1006,7 +1137,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (!ok) break;
-            if (!epilogue(U.bh, U.i, 1, h * g.subt)) { ok = false; break; }
+            if (!epilogue(U.bh, U.i, 1, h * g.subt, false, 0)) { ok = false; break; }
         }
         // the output stores have completed before the CTA exits
         if (row == 0) bulk_wait_all();

@@ -69,6 +69,8 @@ __device__ __forceinline__ void block_coords(const Geo &g, int j, int &jt, int &
 
 constexpr uint32_t kFlagNonfinite = 0x1u;
 constexpr uint32_t kFlagTimeout = 0x2u;
+// a work list, unit id or list size out of range: the kernel stopped taking units
+constexpr uint32_t kFlagBadWork = 0x4u;
 
 // Workspace header: word 0 is the sticky status word.
 struct WsHeader {

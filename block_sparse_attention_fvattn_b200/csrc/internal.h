@@ -15,8 +15,9 @@ struct WsLayout {
     size_t qbar;         // fp32 [BH, nb, D]   pooled query means ([BH][2][nb, D] TF32 head, rest if tc_scores)
     size_t kbarT;        // fp32 [BH, D, nbp]  pooled key means, transposed ([BH][2][nbp, D] if tc_scores)
     size_t scores;       // fp32 [BH, nb, nbp] block scores (tc_scores only)
-    size_t unit_cost;    // int32 [BH*nb]      scheduler: cost per unit
-    size_t head_sorted;  // int32 [BH*nb]      scheduler: units of each head by cost
+    size_t unit_cost;    // int32 [BH*(nb+npair)] scheduler: cost per unit id (paired split units after the others)
+    size_t head_sorted;  // int32 [BH*(nb+2)]  scheduler: unit ids of each head by cost
+    size_t head_len;     // int32 [BH]         scheduler: units of each head
     size_t head_cost;    // int64 [BH]         scheduler: total cost per head
     size_t pair_cnt;     // int32 [BH*npair]   paired mode: union size of each pair of query blocks
     size_t pair_list;    // int32 [BH*npair*nb] paired mode: the union, ascending, with membership flags
@@ -49,7 +50,7 @@ cudaError_t launch_score_gemm(const Geo &g, const float *qhi, const float *qlo, 
 constexpr int kTcScoresMinBlocks = 320;
 cudaError_t launch_schedule(const Geo &g, const int32_t *kv_cnt, const int32_t *kv_idx, int dense, int num_ctas,
                             int32_t *work, int32_t *cta_range, int64_t *cta_cost, int32_t *unit_cost,
-                            int32_t *head_sorted, int64_t *head_cost, const int32_t *pair_cnt,
+                            int32_t *head_sorted, int32_t *head_len, int64_t *head_cost, const int32_t *pair_cnt,
                             cudaStream_t stream);
 // Paired mode (64-token blocks): entry = block | kPairInA (kept by the first
 // query block of the pair) | kPairInB (kept by the second).

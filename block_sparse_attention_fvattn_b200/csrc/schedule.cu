@@ -144,51 +144,91 @@ __device__ __forceinline__ int pair_tiles(const Geo &g, int bh, int pp, const in
     return (c + 1) >> 1;
 }
 
+// Paired mode: a unit of at least kSplitMinTiles key/value tiles runs split,
+// one unit per pair (both softmax warpgroups on the same 128 query rows, each
+// over half of the pair's key list), so the longest units are half as long
+// and the dynamic order can even out the end of the layer; shorter units keep
+// two pairs (one per warpgroup).
+constexpr int kSplitMinTiles = 64;
+
 __global__ void __launch_bounds__(1024) sched_head_kernel(Geo g, const int32_t *__restrict__ kv_cnt,
                                                           const int32_t *__restrict__ kv_idx, int dense,
                                                           const int32_t *__restrict__ pair_cnt,
                                                           int32_t *__restrict__ unit_cost,
                                                           int32_t *__restrict__ head_sorted,
+                                                          int32_t *__restrict__ head_len,
                                                           int64_t *__restrict__ head_cost, int npow2)
 {
     extern __shared__ unsigned long long keys[];
     __shared__ long long part[32];
+    __shared__ int part_n[32];
     pdl_release();
     pdl_wait();  // kept lists or pair unions from the kernel before
     const int bh = blockIdx.x;
     const int hw = g.nbh * g.nbw;
+    // candidate entries of this head: unpaired, entry i = unit i; paired,
+    // entries 2q and 2q+1 = unit q, or its two pairs as split units
+    const int nent = g.paired ? 2 * g.upb : g.upb;
     long long local = 0;
-    for (int i = threadIdx.x; i < npow2; i += blockDim.x) {
-        if (i < g.upb) {
-            const size_t u = (size_t)bh * g.upb + i;
-            int cost;
+    int nvalid = 0;
+    for (int e = threadIdx.x; e < npow2; e += blockDim.x) {
+        unsigned long long key = ~0ull;
+        if (e < nent) {
+            int cost = -1, uid = -1;
             if (g.paired) {
-                // unit i = pairs 2i (first query tile) and 2i+1 (second)
-                cost = pair_tiles(g, bh, 2 * i, pair_cnt, dense) + pair_tiles(g, bh, 2 * i + 1, pair_cnt, dense);
+                const int q = e >> 1, half = e & 1;
+                const int t0 = pair_tiles(g, bh, 2 * q, pair_cnt, dense);
+                const int t1 = pair_tiles(g, bh, 2 * q + 1, pair_cnt, dense);
+                if (!dense && t0 + t1 >= kSplitMinTiles) {
+                    const int pp = 2 * q + half;
+                    if (pp < g.npair) {
+                        cost = half ? t1 : t0;
+                        uid = g.BH * g.upb + bh * g.npair + pp;
+                    }
+                } else if (half == 0) {
+                    // unit q = pairs 2q (first query tile) and 2q+1 (second)
+                    cost = t0 + t1;
+                    uid = bh * g.upb + q;
+                }
             } else {
-                const int it = i / hw;
+                const size_t u = (size_t)bh * g.upb + e;
+                const int it = e / hw;
                 const int nh = (g.nsub == 2 && it * g.bt + g.subt < g.T) ? 2 : 1;
                 const int cnt = dense ? g.nb : __ldg(kv_cnt + u);
                 cost = nh * unit_tiles(g, dense ? nullptr : kv_idx + u * g.nb, cnt, dense);
+                uid = (int)u;
             }
-            unit_cost[u] = cost;
-            local += cost;
-            keys[i] = ((unsigned long long)(0xFFFFFFFFu - (uint32_t)cost) << 32) | (uint32_t)i;
-        } else {
-            keys[i] = ~0ull;
+            if (uid >= 0) {
+                unit_cost[uid] = cost;
+                local += cost;
+                ++nvalid;
+                key = ((unsigned long long)(0xFFFFFFFFu - (uint32_t)cost) << 32) | (uint32_t)uid;
+            }
         }
+        keys[e] = key;
     }
-    for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xFFFFFFFFu, local, o);
-    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = local;
+    for (int o = 16; o > 0; o >>= 1) {
+        local += __shfl_xor_sync(0xFFFFFFFFu, local, o);
+        nvalid += __shfl_xor_sync(0xFFFFFFFFu, nvalid, o);
+    }
+    if ((threadIdx.x & 31) == 0) {
+        part[threadIdx.x >> 5] = local;
+        part_n[threadIdx.x >> 5] = nvalid;
+    }
     __syncthreads();
     if (threadIdx.x == 0) {
         long long s = 0;
-        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) s += part[w];
+        int n = 0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+            s += part[w];
+            n += part_n[w];
+        }
         head_cost[bh] = s;
+        head_len[bh] = n;
     }
     bitonic_sort_u64(keys, npow2);
-    for (int r = threadIdx.x; r < g.upb; r += blockDim.x)
-        head_sorted[(size_t)bh * g.upb + r] = (int32_t)(keys[r] & 0xFFFFFFFFull);
+    for (int r = threadIdx.x; r < nent; r += blockDim.x)
+        head_sorted[(size_t)bh * nent + r] = keys[r] == ~0ull ? -1 : (int32_t)(keys[r] & 0xFFFFFFFFull);
 }
 
 // First index of CTA c's list when U ranks are dealt in zigzag rounds of C.
@@ -202,15 +242,18 @@ __host__ __device__ __forceinline__ long long zigzag_start(long long c, long lon
 
 __global__ void __launch_bounds__(1024) sched_assign_kernel(Geo g, int C, const int32_t *__restrict__ unit_cost,
                                                             const int32_t *__restrict__ head_sorted,
+                                                            const int32_t *__restrict__ head_len,
                                                             const int64_t *__restrict__ head_cost,
                                                             int32_t *__restrict__ work, int32_t *__restrict__ cta_range,
                                                             int64_t *__restrict__ cta_cost, int hpow2)
 {
     extern __shared__ unsigned long long sa_smem[];
+    __shared__ int chunk_sum[1024];
     pdl_release();
     pdl_wait();  // unit costs from sched_head_kernel
     unsigned long long *hkeys = sa_smem;          // [hpow2]
     unsigned long long *ccost = sa_smem + hpow2;  // [C]
+    int *off = reinterpret_cast<int *>(ccost + C); // [hpow2 + 1]: first rank of each head in head order
     for (int h = threadIdx.x; h < hpow2; h += blockDim.x) {
         if (h < g.BH) {
             const unsigned long long c = (unsigned long long)head_cost[h];
@@ -222,13 +265,39 @@ __global__ void __launch_bounds__(1024) sched_assign_kernel(Geo g, int C, const 
     for (int c = threadIdx.x; c < C; c += blockDim.x) ccost[c] = 0ull;
     __syncthreads();
     bitonic_sort_u64(hkeys, hpow2);
-    const long long U = (long long)g.BH * g.upb;
+    // ranks of each head in head order: an exclusive prefix of the head lengths
+    const int per = (g.BH + (int)blockDim.x - 1) / (int)blockDim.x;
+    const int h0 = (int)threadIdx.x * per;
+    int s = 0;
+    for (int x = h0; x < min(h0 + per, g.BH); ++x) s += __ldg(head_len + (int)(hkeys[x] & 0xFFFFFFFFull));
+    chunk_sum[threadIdx.x] = s;
+    __syncthreads();
+    for (int o = 1; o < (int)blockDim.x; o <<= 1) {
+        const int add = (int)threadIdx.x >= o ? chunk_sum[threadIdx.x - o] : 0;
+        __syncthreads();
+        chunk_sum[threadIdx.x] += add;
+        __syncthreads();
+    }
+    int run = chunk_sum[threadIdx.x] - s;
+    for (int x = h0; x < min(h0 + per, g.BH); ++x) {
+        off[x] = run;
+        run += __ldg(head_len + (int)(hkeys[x] & 0xFFFFFFFFull));
+    }
+    if (threadIdx.x == blockDim.x - 1) off[g.BH] = chunk_sum[blockDim.x - 1];
+    __syncthreads();
+    const long long U = off[g.BH];
+    const int stride = g.paired ? 2 * g.upb : g.upb;
     for (int c = threadIdx.x; c <= C; c += blockDim.x) cta_range[c] = (int32_t)zigzag_start(c, U, C);
     for (long long r = threadIdx.x; r < U; r += blockDim.x) {
-        const long long hr = r / g.upb, local = r - hr * g.upb;
-        const int head = (int)(hkeys[hr] & 0xFFFFFFFFull);
-        const int i = head_sorted[(size_t)head * g.upb + local];
-        const long long u = (long long)head * g.upb + i;
+        // the head whose ranks hold r: the last x with off[x] <= r
+        int lo = 0, hi = g.BH - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (off[mid] <= r) lo = mid;
+            else hi = mid - 1;
+        }
+        const int head = (int)(hkeys[lo] & 0xFFFFFFFFull);
+        const int u = head_sorted[(size_t)head * stride + (r - off[lo])];
         const long long round = r / C, pos = r - round * C;
         const long long c = (round & 1) ? (C - 1 - pos) : pos;
         work[zigzag_start(c, U, C) + round] = (int32_t)u;
@@ -248,23 +317,23 @@ static int next_pow2(int n)
 
 cudaError_t launch_schedule(const Geo &g, const int32_t *kv_cnt, const int32_t *kv_idx, int dense, int num_ctas,
                             int32_t *work, int32_t *cta_range, int64_t *cta_cost, int32_t *unit_cost,
-                            int32_t *head_sorted, int64_t *head_cost, const int32_t *pair_cnt,
+                            int32_t *head_sorted, int32_t *head_len, int64_t *head_cost, const int32_t *pair_cnt,
                             cudaStream_t stream)
 {
-    const int npow2 = next_pow2(g.upb);
+    const int npow2 = next_pow2(g.paired ? 2 * g.upb : g.upb);
     const size_t smem_a = (size_t)npow2 * sizeof(unsigned long long);
     cudaError_t err = cudaFuncSetAttribute(sched_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a);
     if (err != cudaSuccess) return err;
     err = launch_dependent(sched_head_kernel, dim3(g.BH), dim3(1024), smem_a, stream, g, kv_cnt, kv_idx, dense,
-                           pair_cnt, unit_cost, head_sorted, head_cost, npow2);
+                           pair_cnt, unit_cost, head_sorted, head_len, head_cost, npow2);
     if (err != cudaSuccess) return err;
     const int hpow2 = next_pow2(g.BH);
-    const size_t smem_b = ((size_t)hpow2 + num_ctas) * sizeof(unsigned long long);
+    const size_t smem_b = ((size_t)hpow2 + num_ctas) * sizeof(unsigned long long) + ((size_t)hpow2 + 1) * sizeof(int);
     err = cudaFuncSetAttribute(sched_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b);
     if (err != cudaSuccess) return err;
     return launch_dependent(sched_assign_kernel, dim3(1), dim3(1024), smem_b, stream, g, num_ctas,
-                            (const int32_t *)unit_cost, (const int32_t *)head_sorted, (const int64_t *)head_cost,
-                            work, cta_range, cta_cost, hpow2);
+                            (const int32_t *)unit_cost, (const int32_t *)head_sorted, (const int32_t *)head_len,
+                            (const int64_t *)head_cost, work, cta_range, cta_cost, hpow2);
 }
 
 }  // namespace fvattn

@@ -19,7 +19,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libfvattn.so")
 
 OK, INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA_ERR, NONFINITE, TIMEOUT = range(7)
-FLAG_NONFINITE, FLAG_TIMEOUT = 0x1, 0x2
+FLAG_NONFINITE, FLAG_TIMEOUT, FLAG_BAD_WORK = 0x1, 0x2, 0x4
 
 
 class FVAttnError(RuntimeError):

@@ -84,6 +84,10 @@ typedef enum fvattn_status {
 /* Device status word bits (as returned, combined, by fvattn_read_device_status). */
 #define FVATTN_FLAG_NONFINITE 0x1u
 #define FVATTN_FLAG_TIMEOUT 0x2u
+/* a schedule entry, unit id or list size was out of range (work lists not
+ * made by fvattn_schedule for this problem, or corrupted): the attention
+ * kernel stopped taking units and part of `out` is not written */
+#define FVATTN_FLAG_BAD_WORK 0x4u
 
 /* Element type of Q, K, V and O (the FastVideo VSA backend accepts both,
  * zskr.cn guide, section 5). */

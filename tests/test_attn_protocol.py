@@ -9,6 +9,10 @@ copies and MMA commits as in the kernel, for paired (two query tiles with
 their own key/value streams) and 128-row (both halves share each key/value
 tile) units, and runs them under random interleavings, with TMA copies
 completing in any order and each issuer's MMAs completing in issue order.
+Paired units may be split: both query halves hold the same query rows and
+walk the two halves of one key list; the second half publishes its row
+maxima and sums and hands its Q buffer back, and the first half reads the
+second half's O, combines and stores.
 It checks that:
 - every wait targets the phase the kernel means (its parity never aliases a
   phase two away, in either direction) and that no run deadlocks;
@@ -79,6 +83,8 @@ class Model:
             "UFull": [B(f"UFull{i}") for i in range(SLOTS)],
             "UEmpty": [B(f"UEmpty{i}", 6) for i in range(SLOTS)],   # producer, V, QK, PV, 2 softmax
             "Taken": B("Taken"),
+            "Comb": B("Comb"),
+            "OStaged": [B("OStaged0"), B("OStaged1")],
         }
         self.slots = [None] * SLOTS
         self.next_unit = 0
@@ -89,7 +95,9 @@ class Model:
         self.S = "free"          # free -> writing -> full(h) -> free
         self.P = ["free", "free"]
         self.O = ["free", "free"]  # free -> acc -> complete -> free
+        self.comb = "free"         # the second half's row maxima and sums of a split unit
         self.qk_inflight = [0, 0]
+        self.combs = 0            # split units combined so far (the first half's Comb waits)
         self.async_tma = []       # (callback) completing in any order
         self.fifo = {"qk": [], "pv": [], "st0": [], "st1": []}
 
@@ -291,6 +299,7 @@ class Model:
 
     def softmax(self, h):
         sf, pw, of, n = 0, 0, 0, 0
+        staged = 0                # epilogues of this half that staged and stored a tile
         while True:
             u = yield from self.take(n)
             n += 1
@@ -311,10 +320,35 @@ class Model:
                 self.P[h] = "full"
                 yield ("arrive", self.b["PFull"][h])
                 pw += 1
+            split = self.paired and len(u) > 2 and u[2]
+            if split and h == 1:
+                # second half of a split unit: O_1 complete, row maxima and sums
+                # published, Q[1] handed back; O_1 is read by the first half
+                yield ("wait", self.b["OFull"][1], of)
+                of += 1
+                self.need(self.O[1] == "complete", f"split half 1 ends with O in state {self.O[1]}")
+                self.need(self.comb == "free", f"split half 1 overwrites the combine data ({self.comb})")
+                self.comb = "written"
+                yield ("arrive", self.b["Comb"])
+                self.need(self.Q[1] == "ready" and self.qk_inflight[1] == 0,
+                          f"split half 1 hands back Q[1] in state {self.Q[1]} with {self.qk_inflight[1]} QK in flight")
+                self.Q[1] = "free"
+                yield ("arrive", self.b["QEmpty"][1])
+                continue
             # epilogue: O read, staged in Q[h], stored, Q[h] handed back
             yield ("wait", self.b["OFull"][h], of)
             of += 1
             self.need(self.O[h] == "complete", f"epilogue {h} reads O in state {self.O[h]}")
+            if split and u[1] > 0:
+                # combine: the second half's maxima and sums, then its O
+                yield ("wait", self.b["Comb"], self.combs)
+                self.combs += 1
+                self.need(self.comb == "written", f"combine reads the second half's data in state {self.comb}")
+                self.need(self.O[1] == "complete", f"combine reads O[1] in state {self.O[1]}")
+                self.comb = "free"
+                self.O[1] = "free"
+                if self.mut != "no_comb_release":
+                    yield ("arrive", self.b["OEmpty"][1])
             self.O[h] = "free"
             yield ("arrive", self.b["OEmpty"][h])
             self.need(self.Q[h] == "ready" and self.qk_inflight[h] == 0,
@@ -327,6 +361,10 @@ class Model:
             st.append(read_done)
             if self.mut == "early_q_release":
                 yield ("arrive", self.b["QEmpty"][h])   # before the stores have read the tile
+            # all rows staged: the storing thread waits for this epilogue's phase
+            yield ("arrive", self.b["OStaged"][h])
+            yield ("wait", self.b["OStaged"][h], (of - 1) if self.mut == "staged_phase_from_of" else staged)
+            staged += 1
             yield ("drain", f"st{h}")
             self.need(self.Q[h] == "stored", f"Q[{h}] handed back in state {self.Q[h]}")
             self.Q[h] = "free"
@@ -379,12 +417,18 @@ class Model:
         raise ProtocolError("no progress within the step limit")
 
 
-def random_units(rng, paired, n):
+def random_units(rng, paired, n, split_share=0.0):
     units = []
     for _ in range(n):
         if paired:
             a = rng.randint(1, 4)
             b = rng.choice([0] + [rng.randint(1, 4)] * 5)   # an empty second tile now and then
+            if rng.random() < split_share:
+                # split: the key list's tiles divided, the first half takes the larger part
+                t = rng.randint(1, 8)
+                a, b = (t + 1) // 2, t // 2
+                units.append((a, b, 1))
+                continue
             units.append((a, b))
         else:
             units.append((rng.randint(1, 5), rng.choice([0, 1, 1, 1])))  # (key tiles, has a second half)
@@ -396,6 +440,41 @@ def test_protocol_has_no_deadlock_or_hazard(paired):
     rng = random.Random(1234 + paired)
     for trial in range(150):
         Model(random_units(rng, paired, rng.randint(1, 14)), paired).run(rng)
+
+
+@pytest.mark.parametrize("share", [0.5, 1.0])
+def test_split_units_have_no_deadlock_or_hazard(share):
+    rng = random.Random(4321 + int(share * 10))
+    for trial in range(200):
+        Model(random_units(rng, True, rng.randint(1, 14), share), True).run(rng)
+
+
+def test_staged_phase_counts_only_stored_epilogues():
+    # the second half of a split unit completes O_1 without staging a tile, so
+    # the storing thread's wait must count staged epilogues, not O completions
+    rng = random.Random(13)
+    caught = False
+    for trial in range(300):
+        try:
+            Model(random_units(rng, True, rng.randint(2, 12), 0.6), True, "staged_phase_from_of").run(rng)
+        except ProtocolError:
+            caught = True
+            break
+    assert caught
+
+
+def test_split_units_need_the_combine_release():
+    # the first half of a split unit must hand O_1 back once it has combined,
+    # or the next product into O_1 waits forever
+    rng = random.Random(11)
+    caught = False
+    for trial in range(300):
+        try:
+            Model(random_units(rng, True, rng.randint(2, 12), 0.7), True, "no_comb_release").run(rng)
+        except ProtocolError:
+            caught = True
+            break
+    assert caught
 
 
 @pytest.mark.parametrize("mutation", ["no_q_wait", "no_sfree", "no_pfree", "early_q_release", "no_kempty",
@@ -416,11 +495,15 @@ def test_o_free_wait_is_implied_by_p_order():
     # The PV issuer waits for the epilogue to have read O_h before the next
     # unit's first product into O_h. The model shows that wait never binds:
     # that product needs P_h of the next unit, which the same softmax
-    # warpgroup writes only after its epilogue. The kernel keeps it as a guard.
+    # warpgroup writes only after its epilogue -- and with split units, where
+    # the first half reads O_1, the PV issuer reaches O_1's next product only
+    # after the first half's, whose P comes after the combine. The kernel
+    # keeps the wait as a guard.
     rng = random.Random(7)
-    for trial in range(150):
+    for trial in range(200):
         paired = bool(trial & 1)
-        Model(random_units(rng, paired, rng.randint(1, 14)), paired, "no_o_free").run(rng)
+        share = 0.6 if (paired and trial % 4 == 1) else 0.0
+        Model(random_units(rng, paired, rng.randint(1, 14), share), paired, "no_o_free").run(rng)
 
 
 def test_unit_ring_consumer_count_matches_the_roles():

@@ -95,8 +95,10 @@ def test_outputs_write_nothing_outside_their_extent(wl):
     assert (ix[tail] == SENT_I32).all(), "kv_idx written past kv_cnt"
     assert (ix[~tail] != SENT_I32).all()
     w = work.cpu().numpy()
-    assert (w[BH * units:] == SENT_I32).all(), "work written past the unit count"
-    assert np.array_equal(np.sort(w[:BH * units]), np.arange(BH * units))
+    U = int(rng[C].item())          # units of the schedule (long 64-token units may run split)
+    assert U >= BH * units
+    assert (w[U:] == SENT_I32).all(), "work written past the unit count"
+    assert len(set(w[:U].tolist())) == U
     assert not torch.isnan(probs).any()
     o = out.view(torch.int16).cpu().numpy()
     assert (o != s16).all(), "a valid output element was left unwritten"

@@ -137,6 +137,24 @@ def test_paired_output_independent_of_cta_count_and_schedule(num_ctas):
     assert torch.equal(out2, ref)
 
 
+@pytest.mark.parametrize("num_ctas", [1, 5, 148])
+def test_split_units_independent_of_cta_count(num_ctas):
+    # near-dense 64-token heads run split units; the result must not depend on
+    # which CTA runs which unit
+    wl = gen.custom("split_ctas", 1, 3, 128, (16, 16, 16), (4, 4, 4), 0.95, 4, sigma=2.0,
+                    a_fixed=(0.25, 0.25, 6.0), seed=45)
+    q, k, v = fvtest.make_on_gpu(wl)
+    ref = _engine(wl, num_ctas=148)
+    o_ref = ref(q, k, v).clone()
+    eng = _engine(wl, num_ctas=num_ctas)
+    out = eng(q, k, v)
+    torch.cuda.synchronize()
+    assert eng.status() == 0
+    U = int(eng.cta_range[num_ctas].item())
+    assert U > 3 * 16, "no unit ran split"
+    assert torch.equal(out, o_ref)
+
+
 @pytest.mark.parametrize("groups", [1, 3, 4])
 def test_host_pipeline_matches_device_path(groups):
     # host-resident tensors, copies overlapped with compute per group of heads:

@@ -33,6 +33,13 @@ SMALL = [
     # 128-token (2,8,8) blocks, ragged along every axis: one 128-row query tile per unit
     gen.custom("blk128_ragged", 1, 3, 128, (7, 20, 28), (2, 8, 8), 0.9, 3, sigma=2.0, a_range=(0.5, 4.0), seed=28),
     gen.custom("blk128_d64", 2, 2, 64, (8, 16, 24), (2, 8, 8), 0.85, 2, sigma=1.5, a_range=(0.5, 3.0), seed=29),
+    # near-dense 64-token heads: units of >= 64 tiles run split (one pair on both
+    # softmax warpgroups, combined at the end); the third head stays sparse
+    gen.custom("blk64_split", 1, 3, 128, (16, 16, 16), (4, 4, 4), 0.95, 4, sigma=2.0, a_fixed=(0.25, 0.25, 6.0),
+               seed=30),
+    # split units with ragged edge blocks, D = 64, an even and an odd pair count per unit row
+    gen.custom("blk64_split_ragged_d64", 1, 2, 64, (13, 16, 18), (4, 4, 4), 0.95, 3, sigma=2.0,
+               a_fixed=(0.25, 0.3), seed=31),
 ]
 FULL = [gen.WORKLOADS[n] for n in gen.WORKLOAD_ORDER]
 
@@ -44,36 +51,48 @@ def _oracle_route(orc, wl, q, k):
     return g, qb, kb, r
 
 
-def _units_per_head(wl, nb):
-    """64-token blocks run four query blocks per unit; the other routes one."""
-    bt, bh, bw = wl.block
-    return -(-nb // 4) if bt * bh * bw == 64 else nb
+# A paired unit of at least this many key/value tiles runs as one split unit
+# per pair (the scheduler's threshold).
+SPLIT_MIN_TILES = 64
 
 
-def _host_costs(wl, nb, kv_cnt, kv_idx):
-    """Cost of every unit as the scheduler defines it, recomputed on the host:
-    active 128-row query tiles x kept key/value sub-tiles. With 64-token blocks
-    a unit is query blocks 4q..4q+3: pairs (4q, 4q+1) and (4q+2, 4q+3), each
-    one 128-row tile over the union of its two lists, two blocks per step."""
+def _host_units(wl, nb, kv_cnt, kv_idx):
+    """Every head's units as the scheduler defines them, recomputed on the
+    host: (list per head of (unit id, cost), where the cost is the active
+    128-row query tiles x kept key/value sub-tiles). With 64-token blocks a
+    unit is query blocks 4q..4q+3: pairs (4q, 4q+1) and (4q+2, 4q+3), each one
+    128-row tile over the union of its two lists, two blocks per step; a unit
+    of at least SPLIT_MIN_TILES steps becomes one split unit per pair, with
+    id B*H*upb + bh*npair + pair."""
     T, Hg, W = wl.grid
     bt, bh, bw = wl.block
     nbh, nbw = -(-Hg // bh), -(-W // bw)
     BH = wl.B * wl.H
     cnt = kv_cnt.reshape(BH, nb)
     idx = kv_idx.reshape(BH, nb, nb)
+    heads = []
     if bt * bh * bw == 64:
-        upb = _units_per_head(wl, nb)
-        cost = np.zeros((BH, upb), dtype=np.int64)
+        upb, npair = -(-nb // 4), -(-nb // 2)
+
+        def tiles(h, pp):
+            if pp >= npair:
+                return 0
+            kept = set(idx[h, 2 * pp, :cnt[h, 2 * pp]].tolist())
+            if 2 * pp + 1 < nb:
+                kept |= set(idx[h, 2 * pp + 1, :cnt[h, 2 * pp + 1]].tolist())
+            return (len(kept) + 1) // 2
         for h in range(BH):
+            units = []
             for q in range(upb):
-                for a in (4 * q, 4 * q + 2):
-                    if a >= nb:
-                        continue
-                    kept = set(idx[h, a, :cnt[h, a]].tolist())
-                    if a + 1 < nb:
-                        kept |= set(idx[h, a + 1, :cnt[h, a + 1]].tolist())
-                    cost[h, q] += (len(kept) + 1) // 2
-        return cost
+                t0, t1 = tiles(h, 2 * q), tiles(h, 2 * q + 1)
+                if t0 + t1 >= SPLIT_MIN_TILES:
+                    for half, tc in ((0, t0), (1, t1)):
+                        if 2 * q + half < npair:
+                            units.append((BH * upb + h * npair + 2 * q + half, tc))
+                else:
+                    units.append((h * upb + q, t0 + t1))
+            heads.append(units)
+        return heads
     two = bt * bh * bw == 256
     subt = bt // 2 if two else bt
 
@@ -83,19 +102,18 @@ def _host_costs(wl, nb, kv_cnt, kv_idx):
 
     ns = np.array([nsub(j) for j in range(nb)])
     nh = np.array([1 + (1 if two and (i // (nbh * nbw)) * bt + subt < T else 0) for i in range(nb)])
-    cost = np.zeros((BH, nb), dtype=np.int64)
     for h in range(BH):
-        for i in range(nb):
-            cost[h, i] = nh[i] * ns[idx[h, i, :cnt[h, i]]].sum()
-    return cost
+        heads.append([(h * nb + i, int(nh[i] * ns[idx[h, i, :cnt[h, i]]].sum())) for i in range(nb)])
+    return heads
 
 
-def _expected_work(cost, C):
-    BH, nb = cost.shape
-    heads = sorted(range(BH), key=lambda h: (-cost[h].sum(), h))
+def _expected_work(heads, C):
+    """Heads by total cost descending (ties: lower head), each head's units by
+    cost descending (ties: lower id), ranks dealt to the CTAs in zigzag rounds."""
+    order = sorted(range(len(heads)), key=lambda h: (-sum(c for _, c in heads[h]), h))
     ranked = []
-    for h in heads:
-        ranked += [h * nb + i for i in sorted(range(nb), key=lambda i: (-cost[h, i], i))]
+    for h in order:
+        ranked += [u for u, _ in sorted(heads[h], key=lambda x: (-x[1], x[0]))]
     lists = [[] for _ in range(C)]
     for r, u in enumerate(ranked):
         rd, pos = divmod(r, C)
@@ -138,16 +156,16 @@ def _run(wl, full_rows, dtype=torch.bfloat16):
     C = eng.num_ctas
     work = eng.work.cpu().numpy()
     rng = eng.cta_range.cpu().numpy()
-    U = wl.B * wl.H * _units_per_head(wl, nb)
+    heads = _host_units(wl, nb, cnt, idx)
+    cost = {u: c for units in heads for u, c in units}
+    U = len(cost)
     assert rng[0] == 0 and rng[C] == U and (np.diff(rng) >= 0).all()
-    assert np.array_equal(np.sort(work[:U]), np.arange(U))
-    cost = _host_costs(wl, nb, cnt, idx)
-    expect = _expected_work(cost, C)
+    assert sorted(work[:U].tolist()) == sorted(cost)
+    expect = _expected_work(heads, C)
     for c in range(C):
         assert work[rng[c]:rng[c + 1]].tolist() == expect[c], c
     cta_cost = eng.cta_cost.cpu().numpy()
-    flat = cost.reshape(-1)
-    assert all(cta_cost[c] == flat[work[rng[c]:rng[c + 1]]].sum() for c in range(C))
+    assert all(cta_cost[c] == sum(cost[u] for u in work[rng[c]:rng[c + 1]]) for c in range(C))
     ns = eng.cta_ns.cpu().numpy()
     assert (ns[np.diff(rng) > 0] > 0).all()
 
