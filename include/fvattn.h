@@ -160,8 +160,12 @@ FVATTN_API fvattn_status fvattn_route(const fvattn_problem *prob, const void *q,
  * it. With 64-token blocks the attention runs query blocks (2p, 2p+1) as one
  * 128-row tile over the union of their two kept lists, two key blocks per
  * step; a unit is then four query blocks 4q .. 4q+3 (two such tiles), its id
- * u = (b*H + h)*ceil(nb/4) + q, and its cost the two tiles' steps. For that
- * case this call also writes the unions into the workspace, where
+ * u = (b*H + h)*ceil(nb/4) + q, and its cost the two tiles' steps. A unit of
+ * at least 64 steps is split (not in dense mode): it becomes one unit per
+ * pair p, id B*H*ceil(nb/4) + (b*H + h)*ceil(nb/2) + p, which both halves of
+ * the attention kernel run over the two halves of the pair's union, so the
+ * longest units are half as long. The number of units is cta_range[num_ctas].
+ * For that case this call also writes the unions into the workspace, where
  * fvattn_sparse_attn reads them: give both calls the same workspace. Units are ordered heads by total cost descending, then units within a
  * head by cost descending (ties: lower index); rank r goes to CTA
  * zigzag(r) = r mod 2C < C ? r mod C : 2C-1 - r mod C, so each round of C
@@ -175,7 +179,8 @@ FVATTN_API fvattn_status fvattn_route(const fvattn_problem *prob, const void *q,
  *   dense           nonzero: schedule the all-blocks problem
  *   num_ctas        persistent CTAs (0 = SM count)
  *   work            out int32 [B*H*nb]    unit ids u = (b*H + h)*nb + i, grouped by CTA
- *                                         (64-token blocks: the first B*H*ceil(nb/4) entries)
+ *                                         (64-token blocks: the ids above; the first
+ *                                         cta_range[num_ctas] entries are written)
  *   cta_range       out int32 [num_ctas+1] CTA c runs work[cta_range[c] .. cta_range[c+1])
  *   cta_cost        out int64 [num_ctas]  predicted cost per CTA, or NULL
  */
