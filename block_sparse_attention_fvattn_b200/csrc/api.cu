@@ -310,6 +310,25 @@ fvattn_status fvattn_augment(const fvattn_problem *prob, const float *block_prob
     return FVATTN_OK;
 }
 
+fvattn_status fvattn_set_wait_limit(void *ws, size_t ws_bytes, uint64_t limit_ns, fvattn_stream_t stream)
+{
+    if (!ws || ws_bytes < sizeof(WsHeader) || !aligned16(ws)) return FVATTN_ERR_WORKSPACE;
+    if (launch_header_write(static_cast<uint32_t *>(ws), kHdrWaitLimit, limit_ns, (cudaStream_t)stream) !=
+        cudaSuccess)
+        return FVATTN_ERR_CUDA;
+    return FVATTN_OK;
+}
+
+fvattn_status fvattn_test_withhold_unit(void *ws, size_t ws_bytes, int32_t rank, fvattn_stream_t stream)
+{
+    if (!ws || ws_bytes < sizeof(WsHeader) || !aligned16(ws)) return FVATTN_ERR_WORKSPACE;
+    if (rank < -1) return FVATTN_ERR_INVALID_ARG;
+    if (launch_header_write(static_cast<uint32_t *>(ws), -kHdrWithhold, (uint64_t)(uint32_t)(rank + 1),
+                            (cudaStream_t)stream) != cudaSuccess)
+        return FVATTN_ERR_CUDA;
+    return FVATTN_OK;
+}
+
 fvattn_status fvattn_read_device_status(void *ws, fvattn_stream_t stream, uint32_t *flags)
 {
     if (!ws || !flags) return FVATTN_ERR_INVALID_ARG;

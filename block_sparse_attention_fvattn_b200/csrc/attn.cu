@@ -426,6 +426,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // launched as a programmatic dependent of the scheduler: everything above
     // overlaps its tail; lists, work and counters are read only after this
     pdl_wait();
+    // the wait limit of this call (workspace header, written on the stream before)
+    if (threadIdx.x == 0) wait_limit_setup(abort_flag, status);
+    __syncthreads();
     const uint64_t t_start = globaltimer_ns();
 
     // Units are taken dynamically, longest first, from a counter shared by all
@@ -457,6 +460,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // unit, and a CTA commits to its next unit only as late as the dynamic
         // longest-first order needs.
         bool ok = true;
+        // test word of the workspace header: withhold rank (word - 1), so this
+        // CTA's roles wait for a unit that never comes
+        const long long withhold = (long long)*reinterpret_cast<volatile uint32_t *>(status + kHdrWithhold) - 1;
         for (int n = 0; ok; ++n) {
             const int slot = n % kUnitSlots;
             if (n > 0 && !mbar_wait(bar(L::bTaken), (uint32_t)(n - 1) & 1u, abort_flag)) break;
@@ -464,6 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 !mbar_wait(bar(L::bUEmpty + slot), (uint32_t)((n / kUnitSlots) - 1) & 1u, abort_flag))
                 break;
             const long long r = (long long)atomicAdd(unit_cursor, 1u);
+            if (r == withhold) break;  // nothing is published for this rank
             int u = r < n_units ? rank_to_unit(r, work, cta_range) : -1;
             // a unit id out of range, or a CTA busy far beyond any real layer
             // (20 s), ends this CTA's units with a flag instead of running on

@@ -332,6 +332,18 @@ cudaError_t launch_augment(const Geo &g, const float *probs, long long budget, i
 
 size_t augment_state_bytes() { return sizeof(AugState); }
 
+__global__ void header_write_kernel(uint32_t *header, int word, uint64_t value)
+{
+    if (word >= 0) *reinterpret_cast<uint64_t *>(header + word) = value;
+    else header[-word] = (uint32_t)value;
+}
+
+cudaError_t launch_header_write(uint32_t *header, int word, uint64_t value, cudaStream_t stream)
+{
+    header_write_kernel<<<1, 1, 0, stream>>>(header, word, value);
+    return cudaGetLastError();
+}
+
 }  // namespace fvattn
 
 // ---------------------------------------------------------------------------

@@ -72,11 +72,16 @@ constexpr uint32_t kFlagTimeout = 0x2u;
 // a work list, unit id or list size out of range: the kernel stopped taking units
 constexpr uint32_t kFlagBadWork = 0x4u;
 
-// Workspace header: word 0 is the sticky status word.
+// Workspace header: word 0 is the sticky status word; words 1-2 the attention
+// kernel's unit counter and finished-CTA count; words 4-5 the per-call wait
+// limit in ns (0: kWaitLimitNs); word 6 a test word (r + 1: the attention
+// kernel's unit claimer withholds rank r, so its CTA's waits run out).
 struct WsHeader {
     uint32_t status;
     uint32_t pad[63];
 };
+constexpr int kHdrWaitLimit = 4;  // uint64 at words 4-5
+constexpr int kHdrWithhold = 6;
 
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
@@ -150,6 +155,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 // raises the timeout flag and winds down instead of hanging the GPU.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
+// A kernel's abort flag (int) is followed in shared memory by its wait limit
+// in ns (uint64 at the next 8-byte slot), set up from the workspace header.
+__device__ __forceinline__ void wait_limit_setup(volatile int *abort_flag, const uint32_t *ws_header)
+{
+    const uint64_t lim = *reinterpret_cast<const volatile uint64_t *>(ws_header + kHdrWaitLimit);
+    *reinterpret_cast<volatile uint64_t *>(abort_flag + 2) = lim ? lim : kWaitLimitNs;
+}
+
 // Wait for phase `parity` of `bar`. Returns false if `abort_flag` (shared
 // memory) is raised by another role or the time limit runs out (then it raises
 // `abort_flag` itself).
@@ -157,12 +170,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
+    const uint64_t limit = *reinterpret_cast<volatile uint64_t *>(abort_flag + 2);
     uint32_t n = 0;
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((++n & 15u) == 0) {
             if (*abort_flag) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit) {
                 *abort_flag = 1;
                 return false;
             }

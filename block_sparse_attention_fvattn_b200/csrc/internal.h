@@ -70,5 +70,8 @@ cudaError_t launch_augment(const Geo &g, const float *probs, long long budget, i
                            void *state, long long *row_tie, unsigned long long *added_cost, double *added_mass,
                            cudaStream_t stream);
 size_t augment_state_bytes();
+// Write a workspace header field on the stream: word >= 0 takes a uint64 at
+// words (word, word+1); word < 0 takes a uint32 at word -word.
+cudaError_t launch_header_write(uint32_t *header, int word, uint64_t value, cudaStream_t stream);
 
 }  // namespace fvattn

@@ -105,6 +105,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     const uint32_t tmem = *tmem_slot;
     pdl_release();
     pdl_wait();  // the pooled means come from the pooling kernel
+    if (threadIdx.x == 0) wait_limit_setup(abort_flag, status);
+    __syncthreads();
 
     if (warp == 0) {
         if (lane == 0) {

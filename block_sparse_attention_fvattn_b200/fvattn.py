@@ -59,6 +59,8 @@ def _load():
         "fvattn_rlb_plan": (i32, [vp, i32, i32, vp, i32, vp, vp]),
         "fvattn_lpt_assign": (i32, [vp, i32, i32, vp, vp]),
         "fvattn_augment": (i32, [P, vp, ctypes.c_int64, vp, vp, vp, vp, vp, sz, vp]),
+        "fvattn_set_wait_limit": (i32, [vp, sz, ctypes.c_uint64, vp]),
+        "fvattn_test_withhold_unit": (i32, [vp, sz, i32, vp]),
         "fvattn_status_string": (ctypes.c_char_p, [i32]),
     }
     for name, (res, args) in sig.items():
@@ -71,7 +73,8 @@ def _load():
 _lib = _load()
 EXPORTED = ("fvattn_num_blocks", "fvattn_default_num_ctas", "fvattn_workspace_size", "fvattn_workspace_init",
             "fvattn_route", "fvattn_route_noalloc", "fvattn_schedule", "fvattn_sparse_attn", "fvattn_read_device_status",
-            "fvattn_status_string", "fvattn_head_cost", "fvattn_rlb_plan", "fvattn_lpt_assign", "fvattn_augment")
+            "fvattn_status_string", "fvattn_head_cost", "fvattn_rlb_plan", "fvattn_lpt_assign", "fvattn_augment",
+            "fvattn_set_wait_limit", "fvattn_test_withhold_unit")
 
 
 def status_string(s: int) -> str:
@@ -240,6 +243,18 @@ def augment(geo: Geometry, block_probs: torch.Tensor, budget: int, kv_cnt: torch
                              _ptr(added_mass, torch.float64, "added_mass"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
                              _stream(stream))
     _check(st, "fvattn_augment")
+
+
+def set_wait_limit(ws: torch.Tensor, limit_ns: int, stream=None):
+    """Time limit (ns) of every wait inside the kernels of later calls on `ws` (0: default 2 s)."""
+    _check(_lib.fvattn_set_wait_limit(_ptr(ws, torch.uint8, "ws"), ws.numel(), int(limit_ns), _stream(stream)),
+           "fvattn_set_wait_limit")
+
+
+def test_withhold_unit(ws: torch.Tensor, rank: int, stream=None):
+    """Failure-path test hook: the next attention call on `ws` withholds unit rank `rank` (-1: off)."""
+    _check(_lib.fvattn_test_withhold_unit(_ptr(ws, torch.uint8, "ws"), ws.numel(), int(rank), _stream(stream)),
+           "fvattn_test_withhold_unit")
 
 
 def read_device_status(ws: torch.Tensor, stream=None) -> int:

@@ -346,6 +346,26 @@ FVATTN_API fvattn_status fvattn_augment(const fvattn_problem *prob, const float 
                                         int32_t *kv_cnt, int32_t *kv_idx, int64_t *added_pairs, double *added_mass,
                                         void *ws, size_t ws_bytes, fvattn_stream_t stream);
 
+/*
+ * fvattn_set_wait_limit -- the time limit of every wait inside the kernels of
+ * later calls on this workspace, in ns (0: the default, 2 s). A wait that runs
+ * out raises FVATTN_FLAG_TIMEOUT; the kernel then lets its copies and products
+ * in flight finish (each with its own bound), frees its tensor memory and
+ * returns, so the context stays usable. fvattn_workspace_init restores the
+ * default. Asynchronous (a one-thread kernel on `stream`).
+ */
+FVATTN_API fvattn_status fvattn_set_wait_limit(void *ws, size_t ws_bytes, uint64_t limit_ns, fvattn_stream_t stream);
+
+/*
+ * fvattn_test_withhold_unit -- a test of the failure path (zskr.cn guide,
+ * section 6: kernel failures surface instead of being masked): the next
+ * fvattn_sparse_attn on this workspace takes rank `rank` of its unit order
+ * but never hands it to its roles, whose waits then run out (see
+ * fvattn_set_wait_limit); that unit's output is not written. -1 turns it off;
+ * fvattn_workspace_init clears it too. Asynchronous.
+ */
+FVATTN_API fvattn_status fvattn_test_withhold_unit(void *ws, size_t ws_bytes, int32_t rank, fvattn_stream_t stream);
+
 /* Synchronise `stream`, return the device status word's flags (FVATTN_FLAG_*)
  * in *flags, and clear them. Returns CUDA on a failed copy. */
 FVATTN_API fvattn_status fvattn_read_device_status(void *ws, fvattn_stream_t stream, uint32_t *flags);
