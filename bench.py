@@ -32,6 +32,7 @@ the same workload; under torchrun only rank 0 runs it.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -668,10 +669,17 @@ def main():
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "f16"], help="element type of Q, K, V and O")
     ap.add_argument("--e2e-groups", type=int, default=8, help="head groups of the host-buffer pipeline")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="keep only the first H heads of the workload (same grid, blocks and input recipe): "
+                         "a slice small enough for a multi-pass ncu capture of a large layer")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     wl = gen.WORKLOADS[args.workload]
+    if args.heads:
+        if not 0 < args.heads <= wl.H:
+            ap.error(f"--heads must be in [1, {wl.H}]")
+        wl = dataclasses.replace(wl, H=args.heads, name=f"{wl.name}_{args.heads}heads")
     world, rank, local = dist_setup(args.gpus)
     try:
         if args.impl == "reference":
