@@ -10,8 +10,10 @@ resident in HBM and larger than L2, so no flush is needed between its
 steps. The default workload
 is the largest single-GPU layer, the 393k-token long video (B=1, H=12,
 D=128, grid 96x64x64, 4x8x8 blocks -> 1536 blocks, p=0.85, k_min=32); the
-other four workloads are measured after it with an L2 flush between steps and
-reported in the same line under "other_workloads". Per-kernel times are
+other four workloads are measured after it and reported in the same line
+under "other_workloads". A buffer of twice the L2 size is written between
+steps only for a layer whose Q, K and V fit in L2 (the tiny case); the
+others' inputs are larger than L2 (201 MB and more). Per-kernel times are
 medians of per-step CUDA events; each workload's routing lists are checked
 against the fp64 oracle (counts of excused rows under "route_parity").
 
@@ -297,6 +299,21 @@ def l2_flusher(dev):
     return torch.empty(max(2 * l2, 1 << 20), dtype=torch.uint8, device=dev)
 
 
+def use_flush(args, wl, dev, headline):
+    """Whether to write an L2-sized buffer between timed steps: `--flush
+    always|never`, or by default (auto) only when a step's inputs (Q, K, V)
+    fit in L2. Larger inputs cannot stay resident in L2 from one step to the
+    next, and the flush's dirty lines would be written back inside the next
+    step's timed routing."""
+    if args.flush == "always":
+        return True
+    if args.flush == "never":
+        return False
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    elem = 2
+    return 3 * wl.B * wl.H * wl.N * wl.D * elem <= l2
+
+
 def route_parity(wl, q, k, cnt, idx):
     """Routing lists of the GPU vs the fp64 oracle under the parity rule of the
     tests (rows identical / excused at the Top-p boundary / excused as rounding
@@ -539,7 +556,8 @@ def run_gpu(args, wl, world, rank, local):
     pk, pk_src = peaks()
     stream = torch.cuda.current_stream()
     fields, total_ms, F, eng, (q, k, v, out), clk, launches, seed = measure(
-        args, wl, dev, rank, world, flush=False, steps=args.steps, warmup=args.warmup, pk=pk, headline=True)
+        args, wl, dev, rank, world, flush=use_flush(args, wl, dev, headline=True), steps=args.steps,
+        warmup=args.warmup, pk=pk, headline=True)
     total_ms_max = max_over_ranks(total_ms, world)
     ms_per_step = total_ms_max / args.steps
     work_all = sum_over_ranks(float(F), world)
@@ -610,7 +628,8 @@ def run_gpu(args, wl, world, rank, local):
     others = {}
     extra = [] if (args.no_extra or world > 1) else [n for n in gen.WORKLOAD_ORDER if n != wl.name]
     for name in extra:
-        f2, _, _, e2, ts, _, _, _ = measure(args, gen.WORKLOADS[name], dev, rank, world, flush=True,
+        w2 = gen.WORKLOADS[name]
+        f2, _, _, e2, ts, _, _, _ = measure(args, w2, dev, rank, world, flush=use_flush(args, w2, dev, headline=False),
                                             steps=min(args.steps, 10), warmup=3, pk=pk, headline=False)
         others[name] = f2
         del e2, ts
@@ -669,6 +688,8 @@ def main():
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "f16"], help="element type of Q, K, V and O")
     ap.add_argument("--e2e-groups", type=int, default=8, help="head groups of the host-buffer pipeline")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
+    ap.add_argument("--flush", default="auto", choices=["auto", "always", "never"],
+                    help="L2 flush between timed steps (auto: only when a step's inputs fit in L2)")
     ap.add_argument("--heads", type=int, default=0,
                     help="keep only the first H heads of the workload (same grid, blocks and input recipe): "
                          "a slice small enough for a multi-pass ncu capture of a large layer")
