@@ -56,17 +56,7 @@
 // paired mode, the two union sizes and the first entries of each union, so no
 // role starts a unit with a chain of global loads.
 #include "common.cuh"
-#include "exp2_poly.h"
 #include "internal.h"
-
-// Pairs of softmax columns (out of every 16) whose exponential is evaluated
-// with the polynomial on the FMA/ALU pipes instead of the MUFU unit. Off by
-// default: measured on B200 the MUFU unit is not the limit of this kernel, and
-// the extra FMA/ALU instructions slow the MMA issue warp that shares their
-// sub-partitions (Wan-5B-like layer: 724 / 687 / 650 TFLOPS for 0 / 4 / 8).
-#ifndef FV_POLY_PAIRS
-#define FV_POLY_PAIRS 0
-#endif
 
 namespace fvattn {
 
@@ -335,31 +325,6 @@ struct UnitFeed {
     }
     __device__ __forceinline__ int meta(int slot, int i) const { return slots[slot * kUnitWords + i]; }
 };
-
-// Two exponentials 2^a (a = packed pair) on the FMA/ALU pipes:
-// a = j + f with j = round(a) (1.5*2^23 rounding constant), f in [-1/2, 1/2],
-// 2^a = 2^j * p(f) with p the degree-3 minimax polynomial of exp2_poly.h; 2^j is
-// applied by adding j to the exponent field. Arguments below -126 give values
-// below 2^-126 (a denormal or zero pattern), never NaN.
-__device__ __forceinline__ void exp2_poly_x2(uint64_t a, float &p0, float &p1)
-{
-    float a0, a1;
-    f2_unpack(a, a0, a1);
-    // p(f) lies in [0.70, 1.42], i.e. its biased exponent is 126 or 127, so adding
-    // j >= -126 to the exponent field can neither wrap nor reach the sign bit
-    a0 = fmaxf(a0, -126.0f);
-    a1 = fmaxf(a1, -126.0f);
-    const float t0 = a0 + 12582912.0f, t1 = a1 + 12582912.0f;  // round to nearest integer
-    const float f0 = a0 - (t0 - 12582912.0f), f1 = a1 - (t1 - 12582912.0f);
-    const uint64_t f = f2_pack(f0, f1);
-    uint64_t q = f2_fma(f2_pack(FV_EXP2_C3, FV_EXP2_C3), f, f2_pack(FV_EXP2_C2, FV_EXP2_C2));
-    q = f2_fma(q, f, f2_pack(FV_EXP2_C1, FV_EXP2_C1));
-    q = f2_fma(q, f, f2_pack(FV_EXP2_C0, FV_EXP2_C0));
-    float q0, q1;
-    f2_unpack(q, q0, q1);
-    p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-    p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
-}
 
 template <int D, int BKV, bool PAIRED, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -862,8 +827,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     l *= alpha;
                 }
             }
-            // p = 2^(x*scale*log2e - m): packed fp32x2 FMA/ADD, MUFU ex2 (or the
-            // polynomial), packed to bf16 pairs in registers first, so this work
+            // p = 2^(x*scale*log2e - m): packed fp32x2 FMA/ADD and MUFU ex2,
+            // packed to bf16 pairs in registers first, so this work
             // overlaps the PV that still reads the previous P_h
             // paired mode: a row whose own query block kept no block of the
             // tiles so far has m = -inf; its p are 0 (not inf - inf)
@@ -876,15 +841,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int q2 = 0; q2 < BKV / 2; ++q2) {
                 const uint64_t a = f2_fma(f2_pack(x[2 * q2], x[2 * q2 + 1]), sl2x2, q2 < BKV / 4 ? neg_a : neg_b);
-                float p0, p1;
-                if ((q2 & 7) < FV_POLY_PAIRS / 2) {
-                    exp2_poly_x2(a, p0, p1);
-                } else {
-                    float a0, a1;
-                    f2_unpack(a, a0, a1);
-                    p0 = ex2_approx(a0);
-                    p1 = ex2_approx(a1);
-                }
+                float a0, a1;
+                f2_unpack(a, a0, a1);
+                const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
                 s4[q2 & 3] = f2_add(s4[q2 & 3], f2_pack(p0, p1));
                 pk[q2] = pack16x2<F16>(p0, p1);
             }
