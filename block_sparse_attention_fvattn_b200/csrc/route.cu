@@ -176,16 +176,20 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geo g, int nxs, cons
 
 // ---------------------------------------------------------------------------
 // K2
-// Query blocks per CTA (rows of the score tile). Each CTA reads its head's
-// whole pooled-key matrix once, so rows longer than 1024 blocks take 16 rows
-// per CTA (two per warp) to halve that traffic; shorter rows take 8 (one per
-// warp) to keep more CTAs in flight.
-template <int EPL>
-constexpr int kSelRowsFor = EPL >= 32 ? 16 : 8;
-// CTAs per SM the register budget is sized for (the score tile and the row's
-// keys live in registers).
-template <int EPL>
-constexpr int kSelMinBlocksFor = EPL >= 32 ? 2 : 3;
+// Query blocks per CTA (rows of the score tile). A CTA that computes its
+// scores (TC false) reads its head's whole pooled-key matrix once, so rows
+// longer than 1024 blocks take 16 rows per CTA (two per warp) to halve that
+// traffic; otherwise 8 (one per warp) keep more CTAs in flight.
+template <int EPL, bool TC>
+constexpr int kSelRowsFor = (!TC && EPL >= 32) ? 16 : 8;
+// CTAs per SM the register budget is sized for: the row's keys live in
+// registers, and so does the score tile when the CTA computes it. With scores
+// from the tensor-core kernel (TC) the tile is only copied, which leaves room
+// for 5 CTAs per SM on rows of up to 512 blocks (48 registers), 4 up to 1024
+// and 3 up to 1536, all without spills.
+template <int EPL, bool TC>
+constexpr int kSelMinBlocksFor =
+    TC ? (EPL >= 64 ? 2 : EPL >= 48 ? 3 : EPL >= 24 ? 4 : 5) : (EPL >= 32 ? 2 : 3);
 // Rows of up to 256 blocks select by a warp sort of their keys; longer rows by
 // a binary search over the key space (fewer passes over the row's elements).
 template <int EPL>
@@ -486,15 +490,16 @@ __device__ __forceinline__ void score_tile(const float *kb, const float *qsT, fl
 }
 
 // The CTA (8 warps) routes query blocks i0 .. i0+ROWS-1 of head bh: scores
-// into shared memory, then each warp selects and compacts whole rows. Shared
-// memory: (D + sel_slices(nbp) * nbp) * ROWS floats.
-template <int D, int EPL>
+// into shared memory (computed here, or with TC copied from the tensor-core
+// kernel's output), then each warp selects and compacts whole rows. Shared
+// memory: (D + S * nbp) * ROWS floats, S = sel_slices(nbp), or 1 with TC.
+template <int D, int EPL, bool TC>
 __device__ __forceinline__ void select_rows(const Geo &g, int bh, int i0, float *sel_smem,
                                             const float *qbar, const float *kbarT, const float *scores, float p,
                                             int k_min, int32_t *__restrict__ kv_cnt, int32_t *__restrict__ kv_idx,
                                             float *__restrict__ probs, uint32_t *__restrict__ status)
 {
-    constexpr int ROWS = kSelRowsFor<EPL>;
+    constexpr int ROWS = kSelRowsFor<EPL, TC>;
     float *qsT = sel_smem;             // [D][ROWS]
     float *sc = sel_smem + D * ROWS;   // [S][ROWS][nbp]; slice 0 ends up holding the scores
     const int nrow = min(ROWS, g.nb - i0);
@@ -504,7 +509,7 @@ __device__ __forceinline__ void select_rows(const Geo &g, int bh, int i0, float 
     // scheduler launch behind this grid, then wait for the pooled means
     pdl_release();
     pdl_wait();
-    if (scores) {
+    if constexpr (TC) {
         // ---- block scores computed on the tensor cores: copy the rows
         const float4 *src = reinterpret_cast<const float4 *>(scores + ((size_t)bh * g.nb + i0) * nbp);
         float4 *dst = reinterpret_cast<float4 *>(sc);
@@ -681,16 +686,16 @@ __device__ __forceinline__ void select_rows(const Geo &g, int bh, int i0, float 
     }
 }
 
-template <int D, int EPL>
-__global__ void __launch_bounds__(256, kSelMinBlocksFor<EPL>) score_select_kernel(Geo g, const float *__restrict__ qbar,
+template <int D, int EPL, bool TC>
+__global__ void __launch_bounds__(256, kSelMinBlocksFor<EPL, TC>) score_select_kernel(Geo g, const float *__restrict__ qbar,
                                                            const float *__restrict__ kbarT, float p, int k_min,
                                                            const float *__restrict__ scores,
                                                            int32_t *__restrict__ kv_cnt, int32_t *__restrict__ kv_idx,
                                                            float *__restrict__ probs, uint32_t *__restrict__ status)
 {
     extern __shared__ __align__(16) float sel_smem[];
-    select_rows<D, EPL>(g, blockIdx.y, blockIdx.x * kSelRowsFor<EPL>, sel_smem, qbar, kbarT, scores, p, k_min, kv_cnt,
-                        kv_idx, probs, status);
+    select_rows<D, EPL, TC>(g, blockIdx.y, blockIdx.x * kSelRowsFor<EPL, TC>, sel_smem, qbar, kbarT, scores, p, k_min,
+                            kv_cnt, kv_idx, probs, status);
 }
 
 // ---------------------------------------------------------------------------
@@ -737,15 +742,16 @@ cudaError_t launch_pool(const Geo &g, const void *q, const void *k, float *qbar,
     return launch_pool_d<64>(g, q, k, qbar, kbarT, stream);
 }
 
-template <int D, int EPL>
-static cudaError_t launch_sel_t(const Geo &g, const float *qbar, const float *kbarT, const float *scores, float p,
-                                int k_min, int32_t *kv_cnt, int32_t *kv_idx, float *probs, uint32_t *status,
-                                cudaStream_t stream, bool programmatic)
+template <int D, int EPL, bool TC>
+static cudaError_t launch_sel_tc(const Geo &g, const float *qbar, const float *kbarT, const float *scores, float p,
+                                 int k_min, int32_t *kv_cnt, int32_t *kv_idx, float *probs, uint32_t *status,
+                                 cudaStream_t stream, bool programmatic)
 {
-    constexpr int ROWS = kSelRowsFor<EPL>;
+    constexpr int ROWS = kSelRowsFor<EPL, TC>;
     // + 32*EPL floats: a row's lanes read positions up to 32*EPL - 1
-    const size_t smem = ((size_t)(D + sel_slices(g.nbp) * g.nbp) * ROWS + 32 * EPL) * sizeof(float);
-    auto kern = score_select_kernel<D, EPL>;
+    const int S = TC ? 1 : sel_slices(g.nbp);
+    const size_t smem = ((size_t)(D + S * g.nbp) * ROWS + 32 * EPL) * sizeof(float);
+    auto kern = score_select_kernel<D, EPL, TC>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     // programmatic dependent launch: the CTAs may be scheduled while the
@@ -756,6 +762,18 @@ static cudaError_t launch_sel_t(const Geo &g, const float *qbar, const float *kb
                                 probs, status);
     kern<<<grid, 256, smem, stream>>>(g, qbar, kbarT, p, k_min, scores, kv_cnt, kv_idx, probs, status);
     return cudaGetLastError();
+}
+
+template <int D, int EPL>
+static cudaError_t launch_sel_t(const Geo &g, const float *qbar, const float *kbarT, const float *scores, float p,
+                                int k_min, int32_t *kv_cnt, int32_t *kv_idx, float *probs, uint32_t *status,
+                                cudaStream_t stream, bool programmatic)
+{
+    if (scores)
+        return launch_sel_tc<D, EPL, true>(g, qbar, kbarT, scores, p, k_min, kv_cnt, kv_idx, probs, status, stream,
+                                           programmatic);
+    return launch_sel_tc<D, EPL, false>(g, qbar, kbarT, scores, p, k_min, kv_cnt, kv_idx, probs, status, stream,
+                                        programmatic);
 }
 
 template <int D>
