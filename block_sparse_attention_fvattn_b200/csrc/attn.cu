@@ -541,6 +541,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int u = um[0];
                 if (u < 0) break;
                 if constexpr (PAIRED) {
+                    // paired units load both Q tiles first: a short unit's first
+                    // products need them before any key tile
                     const PairUnit P = pair_unit_from(g, u, um[1], um[2], pair_list, dense);
                     for (int h = 0; h < 2 && ok && !vrole; ++h) {
                         if (P.cnt(h) == 0) continue;
@@ -567,14 +569,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!vrole) mbar_arrive(bar(L::bTaken));
                     continue;
                 }
-                const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
-                for (int h = 0; h < U.nh && ok && !vrole; ++h) ok = load_q(h, U.i, 1, h * g.subt, U.bh);
-                TileCursor cur;
-                for (int k = 0; k < U.nkv && ok; ++k) {
-                    ok = load_kv(cur.block(U), 0, cur.s * g.subt, U.bh);
-                    cur.advance(g, U);
+                if constexpr (!PAIRED) {
+                    // The first kNK key tiles of a unit go to ring slots last filled
+                    // by the previous unit, so they are issued before this unit's Q
+                    // loads wait for the previous unit's epilogues; a later tile's
+                    // slot frees only after this unit's own first products.
+                    const Unit U = load_unit(g, u, kv_cnt, kv_idx, dense);
+                    const int early = vrole ? 0 : min(U.nkv, L::kNK);
+                    TileCursor cur;
+                    int k = 0;
+                    for (; k < early && ok; ++k) {
+                        ok = load_kv(cur.block(U), 0, cur.s * g.subt, U.bh);
+                        cur.advance(g, U);
+                    }
+                    for (int h = 0; h < U.nh && ok && !vrole; ++h) ok = load_q(h, U.i, 1, h * g.subt, U.bh);
+                    for (; k < U.nkv && ok; ++k) {
+                        ok = load_kv(cur.block(U), 0, cur.s * g.subt, U.bh);
+                        cur.advance(g, U);
+                    }
+                    if (!vrole) mbar_arrive(bar(L::bTaken));
                 }
-                if (!vrole) mbar_arrive(bar(L::bTaken));
             }
             if (!ok) {
                 // wind down: let every copy already issued land before the CTA exits

@@ -148,28 +148,53 @@ class Model:
         self.async_tma.append(done)
 
     def producer(self):
+        """Q and K loads, in the kernel's order. Paired: both Q tiles, then the
+        key tiles. Otherwise a unit's first NK key tiles go to ring slots last
+        filled by the previous unit, so they are issued before the unit's Q
+        loads wait for the previous epilogues (mutation k_ahead: one more,
+        whose slot frees only after this unit's own first product)."""
         kc, qloads, n = 0, [0, 0], 0
+        early = NK + 1 if self.mut == "k_ahead" else NK
         while True:
             u = yield from self.take(n)
             if u is None:
                 return
-            for h in (0, 1):
-                if self.tiles(u, h) == 0:
-                    continue
+
+            def load_q(h):
                 if qloads[h] > 0 and self.mut != "no_q_wait":
                     yield ("wait", self.b["QEmpty"][h], qloads[h] - 1)
                 self.load("Q", h, self.b["QFull"][h])
                 qloads[h] += 1
-            nk = max(u[0], u[1]) if self.paired else u[0]
-            for r in range(nk):
-                for h in ((0, 1) if self.paired else (0,)):
-                    if self.paired and r >= u[h]:
-                        continue
-                    ks = kc % NK
-                    if kc >= NK and self.mut != "no_kempty":
-                        yield ("wait", self.b["KEmpty"][ks], kc // NK - 1)
-                    self.load("K", ks, self.b["KFull"][ks])
-                    kc += 1
+
+            def load_k():
+                nonlocal kc
+                ks = kc % NK
+                if kc >= NK and self.mut != "no_kempty":
+                    yield ("wait", self.b["KEmpty"][ks], kc // NK - 1)
+                self.load("K", ks, self.b["KFull"][ks])
+                kc += 1
+
+            if self.paired:
+                for h in (0, 1):
+                    if u[h]:
+                        yield from load_q(h)
+                for r in range(max(u[0], u[1])):
+                    for h in (0, 1):
+                        if r < u[h]:
+                            yield from load_k()
+            else:
+                q_issued = False
+                for k in range(u[0]):
+                    if not q_issued and k == early:
+                        for h in (0, 1):
+                            if self.tiles(u, h):
+                                yield from load_q(h)
+                        q_issued = True
+                    yield from load_k()
+                if not q_issued:
+                    for h in (0, 1):
+                        if self.tiles(u, h):
+                            yield from load_q(h)
             if self.mut != "no_taken":
                 yield ("arrive", self.b["Taken"])
             n += 1
@@ -489,6 +514,20 @@ def test_planted_protocol_mistakes_are_caught(mutation):
             caught = True
             break
     assert caught, mutation
+
+
+def test_key_loads_ahead_of_q_are_bounded_by_the_ring():
+    # One more early key tile than the ring holds waits for this unit's own
+    # first product, which needs the Q load queued behind it: a deadlock.
+    rng = random.Random(7)
+    caught = False
+    for trial in range(300):
+        try:
+            Model(random_units(rng, False, rng.randint(2, 12)), False, "k_ahead").run(rng)
+        except ProtocolError:
+            caught = True
+            break
+    assert caught
 
 
 def test_o_free_wait_is_implied_by_p_order():
