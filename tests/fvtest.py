@@ -33,9 +33,9 @@ def gamma(n):
     return n * U32 / (1.0 - n * U32)
 
 
-def geometry(wl, dtype=torch.bfloat16):
+def geometry(wl, dtype=torch.bfloat16, softmax_scale=0.0):
     from block_sparse_attention_fvattn_b200 import fvattn as fa
-    return fa.Geometry(wl.B, wl.H, wl.D, wl.grid, wl.block, dtype=dtype)
+    return fa.Geometry(wl.B, wl.H, wl.D, wl.grid, wl.block, softmax_scale=softmax_scale, dtype=dtype)
 
 
 def make_on_gpu(wl, seed=None, dtype=torch.bfloat16):
@@ -270,6 +270,14 @@ def sample_rows(wl, kv_cnt, n_random=96, seed=0):
                 x = min(W - 1, jx * bw + int(rng.integers(bw)))
                 rows.add(int(bhh) * N + (t * Hg + y) * W + x)
     return np.array(sorted(rows), dtype=np.int64)
+
+
+def attn_excess(gpu_out, rows, ref, D, rel):
+    """max over the checked elements of |gpu - ref| - rel * |ref|: the error
+    left after each element's own output rounding (rel = the element type's
+    unit roundoff) is taken off."""
+    got = gpu_out.reshape(-1, D)[torch.from_numpy(rows).to(gpu_out.device)].float().cpu().numpy().astype(np.float64)
+    return float((np.abs(got - ref) - rel * np.abs(ref)).max())
 
 
 def attn_errors(gpu_out, rows, ref, D):

@@ -113,11 +113,11 @@ def pin_pool_ragged_bruteforce(orc):
 
 
 # ---------------------------------------------------------------- routing
-def _route_small(orc, grid, block, p, k_min, H=2, D=32, iid=True, seed=5):
+def _route_small(orc, grid, block, p, k_min, H=2, D=32, iid=True, seed=5, scale=None):
     wl, q, k, v = _small(grid, block, H=H, D=D, iid=iid, seed=seed)
     g = orc.geom(wl.B, wl.H, grid, block, D)
     qb, kb = orc.pool(g, q), orc.pool(g, k)
-    scale = 1.0 / math.sqrt(D)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
     r = orc.route(g, qb, kb, scale, p, k_min)
     return wl, g, q, k, v, qb, kb, scale, r
 
@@ -228,6 +228,34 @@ def pin_route_order_probs_cum(orc):
                 assert r["order"][0, h, i].tolist() == expect.tolist(), (grid, h, i)
         ranked = np.take_along_axis(P, r["order"].astype(np.int64), -1)
         np.testing.assert_allclose(r["cum"], np.cumsum(ranked, axis=-1), rtol=0, atol=1e-12)
+
+
+def pin_custom_scale(orc):
+    """A softmax scale other than 1/sqrt(D) (the problem's softmax_scale
+    override) enters the block scores and the attention logits alike: the
+    probabilities are numpy's softmax of scale * Qbar.Kbar, the attention over
+    the kept lists is SDPA with that scale under the lists' token mask, and
+    the lists differ from those of the default scale (the value is used)."""
+    grid, block, D = (6, 13, 10), (4, 8, 8), 16
+    default = _route_small(orc, grid, block, 0.8, 1, H=2, D=D, iid=False, seed=17)[-1]
+    for scale in (0.9, 0.04):
+        wl, g, q, k, v, qb, kb, sc, r = _route_small(orc, grid, block, 0.8, 1, H=2, D=D, iid=False, seed=17,
+                                                      scale=scale)
+        assert sc == scale
+        np.testing.assert_allclose(r["probs"], _softmax_rows(_np_scores(qb, kb, scale)), rtol=0, atol=1e-13)
+        assert not np.array_equal(r["kv_cnt"], default["kv_cnt"]), scale
+        N, nb = wl.N, orc.num_blocks(g)
+        tb = _token_blocks(grid, block).ravel()
+        out, ws = orc.attn_rows(g, q, k, v, scale, np.arange(wl.H * N), r["kv_cnt"], r["kv_idx"])
+        np.testing.assert_allclose(ws, 1.0, rtol=0, atol=1e-12)
+        for h in range(wl.H):
+            keep = np.zeros((nb, nb), dtype=bool)
+            for i in range(nb):
+                keep[i, r["kv_idx"][0, h, i, :r["kv_cnt"][0, h, i]]] = True
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                q[0, h].double(), k[0, h].double(), v[0, h].double(), attn_mask=torch.from_numpy(keep[tb][:, tb]),
+                scale=scale)
+            np.testing.assert_allclose(out[h * N:(h + 1) * N], ref.numpy(), rtol=0, atol=1e-12)
 
 
 def pin_invariants(orc):
@@ -407,6 +435,6 @@ def pin_fp16_inputs(orc):
 ALL_PINS = [
     pin_vsa_worked_example, pin_long_video_tokens, pin_pool_reshape_mean, pin_pool_ragged_bruteforce,
     pin_topp_bruteforce, pin_topk_reduction, pin_dense_reduction, pin_sparse_attention_masked_sdpa,
-    pin_route_order_probs_cum, pin_invariants, pin_tie_order, pin_nonfinite_repair, pin_element_decode, pin_fp16_inputs,
+    pin_route_order_probs_cum, pin_custom_scale, pin_invariants, pin_tie_order, pin_nonfinite_repair, pin_element_decode, pin_fp16_inputs,
     pin_augment_bruteforce_equal_costs, pin_augment_prefix_rule,
 ]
