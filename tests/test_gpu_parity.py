@@ -248,3 +248,19 @@ MAX_NB = [
 def test_max_block_count_sampled(wl):
     assert math.prod(-(-g // b) for g, b in zip(wl.grid, wl.block)) == 2048
     _run(wl, full_rows=False)
+
+
+# fp16 and D = 64 at layer scale, sampled like the five configurations: the
+# Wan-5B-like layer in fp16, the 64-token layer in fp16, and the Wan-5B-like
+# geometry with 48 heads of D = 64.
+LAYER_VARIANTS = [
+    ("wan5b", torch.float16, None),
+    ("head_skew_64tok", torch.float16, None),
+    ("wan5b_d64", torch.bfloat16, gen.custom("wan5b_d64", 1, 48, 64, (31, 22, 40), (4, 8, 8), 0.9, 8, sigma=2.0,
+                                             a_range=(0.5, 4.0), seed=1002)),
+]
+
+
+@pytest.mark.parametrize("name,dtype,wl", LAYER_VARIANTS, ids=["wan5b-fp16", "head_skew_64tok-fp16", "wan5b_d64"])
+def test_layer_variants_sampled(name, dtype, wl):
+    _run(wl if wl is not None else gen.WORKLOADS[name], full_rows=False, dtype=dtype)
