@@ -4,17 +4,18 @@
 //   video-aware (t,h,w) block (zskr.cn FastVideo VSA guide, section 1: the
 //   post-patch latent grid is cut into spatio-temporal blocks; section 6:
 //   variable-length edge blocks, padding never acts as a key). HBM-bound: one
-//   pass over Q and K with 16-byte coalesced loads; a warp owns one block and
-//   reads its (t, y) runs of contiguous tokens.
+//   pass over Q and K with 16-byte coalesced loads; a CTA pools a strip of one
+//   block row, reading its (t, y) runs of contiguous tokens.
 // K2 score_select_kernel: per (head, query block) row: block scores
 //   s = scale * Qbar_i . Kbar_j, softmax, Top-p with a Top-k floor, diagonal
 //   repair and ascending compaction (ai-feeds.com FVAttn summary, "Key
-//   modules" 1; hotpaper.ai abstract). The nb x nb score matrix never leaves
-//   shared memory. One warp owns one row. Selection is exact in fp32: an
-//   order-preserving integer key of each score and a 4-ary search over the key
-//   space find the score at the Top-p boundary (by probability mass) and, if
-//   the floor binds, at rank m; ties at the boundary go to the lower block
-//   index.
+//   modules" 1; hotpaper.ai abstract). The score rows stay in shared memory
+//   (computed here, or copied from the tensor-core scores of long rows). One
+//   warp owns one row. Selection is exact in fp32 on order-preserving integer
+//   keys of the scores: rows of up to 256 blocks sort their keys; longer rows
+//   bisect the key space to the score at the Top-p boundary (by probability
+//   mass) and, if the floor binds, at rank m. Ties at the boundary go to the
+//   lower block index.
 #include "common.cuh"
 #include "internal.h"
 
