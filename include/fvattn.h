@@ -131,7 +131,7 @@ FVATTN_API fvattn_status fvattn_workspace_init(void *ws, size_t ws_bytes, fvattn
  *   m = min(nb, max(m_p, k_min)); S_i = first m ranked blocks plus block i;
  *   a row with a non-finite score keeps every block and sets FLAG_NONFINITE.
  *
- *   q, k          bf16 [B,H,N,D]
+ *   q, k          [B,H,N,D] in the problem's element type (bf16 or fp16)
  *   p             Top-p threshold, 0 < p <= 1
  *   k_min         Top-k floor, 1 <= k_min <= nb (k_min > nb is INVALID_ARG,
  *                 k_min == nb keeps every block, like VSA's topk rules,
@@ -166,7 +166,8 @@ FVATTN_API fvattn_status fvattn_route(const fvattn_problem *prob, const void *q,
  * the attention kernel run over the two halves of the pair's union, so the
  * longest units are half as long. The number of units is cta_range[num_ctas].
  * For that case this call also writes the unions into the workspace, where
- * fvattn_sparse_attn reads them: give both calls the same workspace. Units are ordered heads by total cost descending, then units within a
+ * fvattn_sparse_attn reads them: give both calls the same workspace.
+ * Units are ordered heads by total cost descending, then units within a
  * head by cost descending (ties: lower index); rank r goes to CTA
  * zigzag(r) = r mod 2C < C ? r mod C : 2C-1 - r mod C, so each round of C
  * consecutive ranks (one head's units run together, which keeps its key/value
