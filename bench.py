@@ -587,13 +587,14 @@ def run_gpu(args, wl, world, rank, local):
     if not args.no_e2e:
         hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
         hout = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
-        pipe = fa.HostPipeline(eng.geo, wl.p, wl.k_min, groups=args.e2e_groups, device=dev)
+        pipe = fa.HostPipeline(eng.geo, wl.p, wl.k_min, groups=args.e2e_groups, device=dev, overlap_calls=True)
         n_e2e = max(2, min(args.steps, 10))
         pipe(hq, hk, hv, hout)
         torch.cuda.synchronize()
         barrier(world)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
+        pipe.restart()  # the first timed call's copies start after `a`
         for _ in range(n_e2e):
             pipe(hq, hk, hv, hout)
         b.record(stream)
@@ -602,7 +603,7 @@ def run_gpu(args, wl, world, rank, local):
         e2e = {"value": work_all / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
                "d2h_bytes_per_step": q.numel() * q.element_size(),
-               "ms_per_step": e2e_ms, "head_groups": len(pipe.ranges)}
+               "ms_per_step": e2e_ms, "head_groups": len(pipe.ranges), "overlap_calls": True}
         del pipe, hq, hk, hv, hout
 
     # ---- the layer's heads split over ranks: emulated on this GPU (N=1), or
@@ -686,7 +687,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "f16"], help="element type of Q, K, V and O")
-    ap.add_argument("--e2e-groups", type=int, default=8, help="head groups of the host-buffer pipeline")
+    ap.add_argument("--e2e-groups", type=int, default=12, help="head groups of the host-buffer pipeline")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
     ap.add_argument("--flush", default="auto", choices=["auto", "always", "never"],
                     help="L2 flush between timed steps (auto: only when a step's inputs fit in L2)")

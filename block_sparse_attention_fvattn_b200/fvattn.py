@@ -352,9 +352,18 @@ class HostPipeline:
     on a third, so a call takes about the host->device copy time plus one
     group's compute and copy-out. The result is the same as FVAttn on the
     whole problem (every head is routed, scheduled and attended alone).
+
+    overlap_calls: by default a call's copies in start only after all work
+    enqueued before it on the current stream, which includes the previous
+    call's last compute and copy-out. With overlap_calls, a call's copy of head
+    group c waits only for the previous call's compute of group c (the reader
+    of those device buffers), so consecutive calls keep the host->device
+    link busy. The host inputs must then be ready when the call is made: no
+    work still pending on a stream may be writing them.
     """
 
-    def __init__(self, geo: Geometry, p: float, k_min: int, groups: int = 4, device="cuda", num_ctas: int = 0):
+    def __init__(self, geo: Geometry, p: float, k_min: int, groups: int = 4, device="cuda", num_ctas: int = 0,
+                 overlap_calls: bool = False):
         BH = geo.B * geo.H
         groups = max(1, min(int(groups), BH))
         self.geo, self.dev = geo, torch.device(device)
@@ -365,6 +374,8 @@ class HostPipeline:
         self.dq, self.dk, self.dv, self.dout = (torch.empty(shape, dtype=geo.dtype, device=self.dev) for _ in range(4))
         self.s_in = torch.cuda.Stream(device=self.dev)
         self.s_out = torch.cuda.Stream(device=self.dev)
+        self.overlap_calls = bool(overlap_calls)
+        self._prev_done = None  # the previous call's compute events, per group
 
     def __call__(self, hq: torch.Tensor, hk: torch.Tensor, hv: torch.Tensor, hout: torch.Tensor):
         """hq, hk, hv, hout: pinned host tensors [B, H, N, D] of the problem's dtype.
@@ -380,11 +391,16 @@ class HostPipeline:
         BH = self.geo.B * self.geo.H
         views = [t.view(BH, self.geo.N, self.geo.D) for t in (hq, hk, hv, hout)]
         compute = torch.cuda.current_stream(self.dev)
-        self.s_in.wait_stream(compute)   # the device buffers are free once earlier work is done
+        prev = self._prev_done if self.overlap_calls else None
+        if prev is None:
+            self.s_in.wait_stream(compute)   # the device buffers are free once earlier work is done
         self.s_out.wait_stream(compute)
         copied, done = [], []
-        for h0, h1 in self.ranges:
+        for c, (h0, h1) in enumerate(self.ranges):
             with torch.cuda.stream(self.s_in):
+                if prev is not None:
+                    # the previous call's compute of this group has read its inputs
+                    self.s_in.wait_event(prev[c])
                 for dst, src in zip((self.dq, self.dk, self.dv), views[:3]):
                     dst[h0:h1].copy_(src[h0:h1], non_blocking=True)
                 ev = torch.cuda.Event()
@@ -401,7 +417,13 @@ class HostPipeline:
                 self.s_out.wait_event(d)
                 views[3][h0:h1].copy_(self.dout[h0:h1], non_blocking=True)
         compute.wait_stream(self.s_out)
+        self._prev_done = done
         return hout
+
+    def restart(self):
+        """Make the next call wait for all work enqueued before it on the
+        current stream, as the first call does (overlap_calls only)."""
+        self._prev_done = None
 
     def status(self) -> int:
         flags = 0

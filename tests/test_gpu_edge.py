@@ -173,6 +173,33 @@ def test_host_pipeline_matches_device_path(groups):
     assert torch.equal(hout, ref.cpu())
 
 
+@pytest.mark.parametrize("groups", [2, 4])
+def test_host_pipeline_overlapped_calls(groups):
+    # overlap_calls: a call's copy of head group c waits only for the previous
+    # call's compute of group c. Three different inputs in a row, no
+    # synchronisation between the calls: each result is bit-identical to the
+    # device path on its own inputs
+    from block_sparse_attention_fvattn_b200 import fvattn as fa
+    wl = gen.custom("host_overlap", 1, 8, 128, (12, 24, 40), (4, 8, 8), 0.9, 4, sigma=2.0, a_range=(0.5, 4.0),
+                    seed=41)
+    eng = _engine(wl)
+    ins, refs = [], []
+    for seed in (41, 42, 43):
+        q, k, v = fvtest.make_on_gpu(wl, seed=seed)
+        refs.append(eng(q, k, v).clone().cpu())
+        ins.append(tuple(t.cpu().pin_memory() for t in (q, k, v)))
+    torch.cuda.synchronize()
+    outs = [torch.zeros(ins[0][0].shape, dtype=ins[0][0].dtype).pin_memory() for _ in ins]
+    pipe = fa.HostPipeline(fvtest.geometry(wl), wl.p, wl.k_min, groups=groups, overlap_calls=True)
+    for (hq, hk, hv), hout in zip(ins, outs):
+        pipe(hq, hk, hv, hout)
+    torch.cuda.synchronize()
+    assert pipe.status() == 0
+    assert not torch.equal(refs[0], refs[1])
+    for hout, ref in zip(outs, refs):
+        assert torch.equal(hout, ref)
+
+
 @pytest.mark.parametrize("block", [(4, 8, 8), (4, 4, 4)])
 def test_cuda_graph_replay_matches_eager(block):
     wl = gen.custom("graph", 1, 3, 128, (9, 20, 28), block, 0.9, 4, sigma=2.0, a_range=(0.5, 4.0), seed=40)
